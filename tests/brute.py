@@ -1,0 +1,132 @@
+"""Brute-force references for the number formats and the Four-Over-Six block
+encoder, written from the format definitions (bit fields) and nearest-value
+search, not from the oracle's decision-point lists.  Test helpers only."""
+import numpy as np
+
+
+def e2m1_from_bits(code: int) -> float:
+    """E2M1 from its bit fields: sign, 2 exponent bits (bias 1), 1 mantissa bit."""
+    s = (code >> 3) & 1
+    e = (code >> 1) & 3
+    m = code & 1
+    v = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1 + m / 2)
+    return -v if s else v
+
+
+def e4m3_from_bits(code: int) -> float:
+    """E4M3 (fn) from its bit fields: 4 exponent bits (bias 7), 3 mantissa bits."""
+    s = (code >> 7) & 1
+    e = (code >> 3) & 15
+    m = code & 7
+    if e == 15 and m == 7:
+        return float("nan")
+    v = (m / 8) * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+    return -v if s else v
+
+
+E2M1_MAGS = np.array(sorted({abs(e2m1_from_bits(c)) for c in range(8)}), np.float64)
+E4M3_POS = np.array([e4m3_from_bits(c) for c in range(0x7F)], np.float64)   # codes 0..0x7E
+
+
+def brute_e2m1(y: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 magnitude by search over all 8 magnitudes; ties to the even
+    magnitude index; sign bit from the input."""
+    # beyond 6 the nearest magnitude is 6 whatever the input; clamping at 8 keeps
+    # the float64 distances exact for huge inputs
+    a = np.minimum(np.abs(y.astype(np.float64)), 8.0)
+    dist = np.abs(a[:, None] - E2M1_MAGS[None, :])
+    best = dist.min(axis=1, keepdims=True)
+    cand = dist == best
+    idx = np.where(cand[:, ::2].any(axis=1),           # prefer an even index on a tie
+                   np.argmax(np.where(cand & (np.arange(8) % 2 == 0), 1, 0), axis=1),
+                   np.argmax(cand, axis=1))
+    sign = np.signbit(y).astype(np.uint8) << 3
+    return (sign | idx.astype(np.uint8)).astype(np.uint8)
+
+
+def brute_e4m3(y: np.ndarray) -> np.ndarray:
+    """Nearest non-negative E4M3 value by search over all 127 finite codes; ties to
+    the even code (mantissa LSB 0).  Above 448 the nearest is 448 (saturation)."""
+    a = np.minimum(np.abs(y.astype(np.float64)), 1024.0)   # exact distances, same nearest
+    out = np.empty(a.shape, np.uint8)
+    for i in range(0, a.size, 1 << 16):
+        blk = a[i:i + (1 << 16)]
+        dist = np.abs(blk[:, None] - E4M3_POS[None, :])
+        best = dist.min(axis=1, keepdims=True)
+        cand = dist == best
+        even = cand & (np.arange(0x7F) % 2 == 0)
+        idx = np.where(even.any(axis=1), np.argmax(even, axis=1), np.argmax(cand, axis=1))
+        out[i:i + (1 << 16)] = idx
+    return out
+
+
+def midpoints_with_neighbours(values: np.ndarray) -> np.ndarray:
+    """Every midpoint between consecutive values, and the fp32 numbers 1 and 2
+    ulps either side of it, plus the values themselves."""
+    v = np.asarray(values, np.float64)
+    mids = ((v[1:] + v[:-1]) / 2).astype(np.float32)
+    pts = [v.astype(np.float32), mids]
+    cur_up, cur_dn = mids.copy(), mids.copy()
+    for _ in range(2):
+        cur_up = np.nextafter(cur_up, np.float32(np.inf))
+        cur_dn = np.nextafter(cur_dn, np.float32(-np.inf))
+        pts += [cur_up.copy(), cur_dn.copy()]
+    return np.concatenate(pts)
+
+
+def e2m1_value(code: np.ndarray) -> np.ndarray:
+    """Decoded E2M1 values (float32) of codes, from the bit fields."""
+    table = np.array([e2m1_from_bits(c) for c in range(16)], np.float32)
+    return table[np.asarray(code, np.uint8) & 15]
+
+
+def e4m3_value(code: np.ndarray) -> np.ndarray:
+    table = np.array([e4m3_from_bits(c) for c in range(256)], np.float32)
+    return table[np.asarray(code, np.uint8)]
+
+
+def four_over_six_blocks(x: np.ndarray, s: np.float32):
+    """Brute-force Four-Over-Six over blocks x [nblocks, 16] (float32) with tensor
+    scale s.  For each target m in (6, 4): the block scale is the nearest E4M3 of
+    amax/(m*s); codes are the nearest E2M1 of x/D (D = scale*s; all +0 if D == 0);
+    the error sums (x - v*D)^2 over elements 0..7 and 8..15 left to right and adds
+    the halves.  Keeps 4 only when its error is strictly lower.
+    Returns (codes [nblocks,16], scale bytes [nblocks], keep4 [nblocks])."""
+    x = np.ascontiguousarray(x, np.float32)
+    s = np.float32(s)
+    amax = np.abs(x).max(axis=1)
+    res = {}
+    for m in (6, 4):
+        ratio = amax / (np.float32(m) * s)
+        sb = brute_e4m3(ratio.astype(np.float32))
+        D = e4m3_value(sb) * s
+        Dc = np.where(D > 0, D, np.float32(1))[:, None]
+        y = (x / Dc).astype(np.float32)
+        q = brute_e2m1(y.reshape(-1)).reshape(x.shape)
+        q = np.where((D > 0)[:, None], q, 0).astype(np.uint8)
+        e = x - e2m1_value(q) * D[:, None]
+        e2 = (e * e).astype(np.float32)
+        lo = e2[:, 0].copy()
+        hi = e2[:, 8].copy()
+        for i in range(1, 8):
+            lo = (lo + e2[:, i]).astype(np.float32)
+            hi = (hi + e2[:, 8 + i]).astype(np.float32)
+        res[m] = (q, sb, (lo + hi).astype(np.float32))
+    keep4 = res[4][2] < res[6][2]
+    codes = np.where(keep4[:, None], res[4][0], res[6][0])
+    sbytes = np.where(keep4, res[4][1], res[6][1])
+    return codes.astype(np.uint8), sbytes.astype(np.uint8), keep4
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """[..., 2j] -> low nibble, [..., 2j+1] -> high nibble of byte j."""
+    c = np.asarray(codes, np.uint8)
+    return (c[..., 0::2] & 15) | ((c[..., 1::2] & 15) << 4)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    p = np.asarray(packed, np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = p & 15
+    out[..., 1::2] = p >> 4
+    return out
