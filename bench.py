@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 KV-cache hot path on B200.
+
+Workload ("layer step", the 5B video DiT shape at 1280x704): one layer of
+streaming generation per step -- NVFP4-quantize the new 7040-token chunk's K
+and V ([7040, 24, 128] bf16) into the cache (K-smoothing, Four-Over-Six),
+evict what left the window, then sink-window attention of the chunk's queries
+Q [7040, 24, 128] over the global sink (chunk 0), the shot sink (chunk 4) and
+the window of 3 chunks: 5 x 7040 = 35,200 keys.  Inputs are seeded synthetic
+tensors (synth/), a rotating pool of 4 (K, V, Q) sets (520 MB, larger than
+the 126 MB L2).
+
+Printed (rank 0, one JSON line): value = sink-window attention TFLOP/s of the
+whole step (4*T_q*L*d*H FLOPs per step over the step's device time, summed
+over ranks); the quantizer's GB/s (algorithmic bytes: bf16 K, V read once,
+codes + scales + mean + tensor scales written once) and both kernels'
+roofline fractions; e2e = the same metric through the public API with host
+buffers (pinned host -> device copies of K, V, Q and the device -> host copy of
+O inside the timed region).
+
+--impl reference times the CPU oracle on a bounded sample of the same step
+(see cpu_baseline in the line).  Multi-GPU: one process per GPU (torchrun),
+independent replicas (no collective on the data path), weak scaling.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+CFG = dict(H=24, d=128, T_c=7040, S_g=1, S_s=1, W=3, seed=2, shot_start=4, prefill=9, pool=4)
+METRIC = "KV quantize GB/s and sink-window attention TFLOP/s (% of roofline), 1 B200"
+WORKLOAD = ("one layer step: NVFP4-quantize K,V [7040,24,128] bf16 into the cache, then "
+            "sink-window attention Q [7040,24,128] over S_g=1, S_s=1, W=3 chunks (35,200 keys)")
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def keys_per_step():
+    return (CFG["S_g"] + CFG["S_s"] + CFG["W"]) * CFG["T_c"]
+
+
+def attn_flops(T_q=None, L=None):
+    T_q = CFG["T_c"] if T_q is None else T_q
+    L = keys_per_step() if L is None else L
+    return 4.0 * T_q * L * CFG["d"] * CFG["H"]
+
+
+def quant_bytes():
+    n = CFG["T_c"] * CFG["H"] * CFG["d"]
+    return 2 * n * 2 + n * 9 // 8 + CFG["H"] * CFG["d"] * 4 + 8
+
+
+def load_peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ our arm
+
+def make_inputs(rank):
+    cfg = dict(CFG, seed=CFG["seed"] + 1000 * rank)
+    return [synth.layer_chunk(cfg, rank, p, T_c=CFG["T_c"], H=CFG["H"], d=CFG["d"])
+            for p in range(CFG["pool"])]
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import sink_window_video_b200 as swv
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    swv.load()
+    host = make_inputs(rank)
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    pool = [tuple(to_dev(x) for x in s) for s in host]
+    pinned = [tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+                    for x in s) for s in host]
+    T, H, d = CFG["T_c"], CFG["H"], CFG["d"]
+    cache = swv.KVCache(1, H, T, CFG["S_g"], CFG["S_s"], CFG["W"])
+    O = torch.empty((T, H, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # fill the cache up to the steady state: chunks 0..8, shot switch at chunk 4
+    for c in range(CFG["prefill"]):
+        if c == CFG["shot_start"]:
+            cache.rebind_shot_sink(c)
+        K, V, _ = pool[c % CFG["pool"]]
+        cache.append(0, K, V)
+    torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        K, V, Q = pool[i % CFG["pool"]]
+        if ev is not None:
+            ev[0].record(stream)
+        cache.append(0, K, V)
+        if ev is not None:
+            ev[1].record(stream)
+        cache.attention(0, Q, O)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert cache.keyset(0) == sorted({0, CFG["shot_start"]} | set(range(
+        cache.num_chunks(0) - CFG["W"], cache.num_chunks(0))))
+    if cache.check_status() != swv.OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_quant = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    ms_attn = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    if cache.check_status() != swv.OK:
+        raise RuntimeError("device status not OK after the timed steps")
+    ms_total = max_over_ranks(ms_total, world)
+
+    # end to end through the public API with host buffers
+    e2e_ms = None
+    if not args.no_e2e:
+        O_host = torch.empty((T, H, d), dtype=torch.bfloat16).pin_memory()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.e2e_steps):
+            Kh, Vh, Qh = pinned[i % CFG["pool"]]
+            K = Kh.to(dev, non_blocking=True)
+            V = Vh.to(dev, non_blocking=True)
+            Q = Qh.to(dev, non_blocking=True)
+            cache.append(0, K, V)
+            cache.attention(0, Q, O)
+            O_host.copy_(O, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+
+    return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
+                e2e_ms=e2e_ms)
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+
+class OracleSample:
+    """The oracle on a bounded sample of the step, prepared once: the float64
+    attention of `rows` query rows of head 0 over the 5 key chunks, and the NVFP4
+    quantization of a `slice_tokens`-token slice of the chunk (all 24 heads).
+    The quantization is per chunk; its cost is prorated to the sampled
+    (row, head) pairs: t_quant_chunk * rows / (7040 * 24)."""
+
+    def __init__(self, rows=32, slice_tokens=704, rank=0):
+        import oracle
+        self.oracle = oracle
+        cfg = dict(CFG, seed=CFG["seed"] + 1000 * rank)
+        K, V, Q = synth.layer_chunk(cfg, rank, 0)
+        K2, V2, _ = synth.layer_chunk(cfg, rank, 1)
+        self.Ks, self.Vs = K[:slice_tokens].copy(), V[:slice_tokens].copy()
+        self.slice_tokens = slice_tokens
+        h = slice(0, 1)
+
+        def head0(q):
+            return dict(q, k_codes=q["k_codes"][h], k_scales=q["k_scales"][h],
+                        k_mean=q["k_mean"][h], v_codes=q["v_codes"][h], v_scales=q["v_scales"][h])
+        old = head0(oracle.quantize_chunk(K2, V2))
+        cur = head0(oracle.quantize_chunk(K, V))
+        self.chunks = [old] * 4 + [cur]
+        self.Q = np.ascontiguousarray(Q[:, h, :])
+        self.rows = np.linspace(0, CFG["T_c"] - 1, rows).astype(np.int32)
+
+    def run(self):
+        t = time.perf_counter()
+        self.oracle.quantize_chunk(self.Ks, self.Vs)
+        tq_chunk = (time.perf_counter() - t) * CFG["T_c"] / self.slice_tokens
+        t = time.perf_counter()
+        self.oracle.attention_f64(self.chunks, self.Q, rows=self.rows)
+        ta = time.perf_counter() - t
+        R = len(self.rows)
+        t_sample = ta + tq_chunk * R / (CFG["T_c"] * CFG["H"])
+        flops = 4.0 * R * keys_per_step() * CFG["d"]
+        return flops / t_sample / 1e12, t_sample, ta, tq_chunk
+
+    def entry(self, value, ta, tq_chunk):
+        return {"value": value, "unit": "TFLOP/s", "cores": self.oracle.get_threads(),
+                "kind": "oracle",
+                "sample": (f"oracle float64 attention of {len(self.rows)} of 7040 query rows, "
+                           f"head 0 of 24, over 35,200 keys ({ta:.3f} s), plus NVFP4 "
+                           f"quantization of a {self.slice_tokens}-token slice of the chunk "
+                           f"scaled to the chunk ({tq_chunk:.3f} s per chunk) and prorated per "
+                           f"(row, head)")}
+
+    def baseline(self, budget_s=12.0):
+        """Repeat the sample for about budget_s seconds; median value."""
+        vals, t0 = [], time.perf_counter()
+        while not vals or time.perf_counter() - t0 < budget_s:
+            v, _, ta, tq = self.run()
+            vals.append(v)
+        return self.entry(statistics.median(vals), ta, tq)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    smp = OracleSample(rows=args.ref_rows)
+    for _ in range(args.warmup):
+        smp.run()
+    vals, times = [], []
+    for _ in range(args.steps):
+        v, ts, ta, tq = smp.run()
+        vals.append(v)
+        times.append(ts)
+    value = statistics.median(vals)
+    entry = smp.entry(value, ta, tq)
+    # ms for one full step at the sampled rate
+    full_ms = 1000.0 * attn_flops() / (value * 1e12)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": full_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded SplitMix64 + Box-Muller, 5B video DiT shapes)",
+            "config": {"workload": WORKLOAD, "sample": entry["sample"],
+                       "sample_seconds_median": statistics.median(times)},
+            "cpu_baseline": entry,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=32)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    r = run_ours(args, rank, world, local)
+    peaks, peak_src = load_peaks()
+    if rank == 0:
+        K = args.steps
+        value = attn_flops() * K * world / (r["ms_total"] / 1e3) / 1e12
+        attn_tf = attn_flops() / (r["ms_attn"] / 1e3) / 1e12
+        quant_gbs = quant_bytes() / (r["ms_quant"] / 1e3) / 1e9
+        tpeak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": r["ms_total"] / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded SplitMix64 + Box-Muller, 5B video DiT shapes)",
+            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": CFG["T_c"],
+                       "keys": keys_per_step(), "heads": CFG["H"], "head_dim": CFG["d"],
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs rotate over 4 sets of K,V,Q (520 MB) > 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": "sink_window_attention",
+                         "achieved": attn_tf, "peak": tpeak, "unit": "TFLOP/s",
+                         "frac": attn_tf / tpeak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 sustained"},
+            "quantize": {"kernel": "nvfp4kv_quantize_chunk", "bound": "hbm",
+                         "achieved": quant_gbs, "peak": hpeak, "unit": "GB/s",
+                         "frac": quant_gbs / hpeak, "bytes_per_launch": quant_bytes(),
+                         "ms_per_launch": r["ms_quant"], "peak_source": f"{peak_src} hbm"},
+            "attention": {"ms_per_launch": r["ms_attn"], "flops_per_launch": attn_flops(),
+                          "tflops": attn_tf},
+            "gpu_launches": 2 * K,
+            "clocks": r["clocks"],
+        }
+        if r["e2e_ms"] is not None:
+            n = CFG["T_c"] * CFG["H"] * CFG["d"]
+            line["e2e"] = {"value": attn_flops() * world / (r["e2e_ms"] / 1e3) / 1e12,
+                           "unit": "TFLOP/s", "h2d_bytes_per_step": 3 * n * 2,
+                           "d2h_bytes_per_step": n * 2, "ms_per_step": r["e2e_ms"]}
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = OracleSample(rows=args.ref_rows).baseline()
+        print(json.dumps(line))
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,267 @@
+/*
+ * nvfp4kv.h -- C ABI of the NVFP4 KV cache and multi-shot sink-window
+ * attention library for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (web pages about LongLive-2.0, arXiv 2605.18739):
+ *   - chunk-level NVFP4 quantization of a video DiT's KV cache, with
+ *     K-smoothing and micro-block scales ("2605-LongLive2" DeepRead page,
+ *     Method > 推理基础设施, parallel KV quantization; tailorednewshub page
+ *     "Infrastruttura Parallela NVFP4", Inferenza W4A4 NVFP4: micro-block
+ *     scaling with Four Over Six scale selection);
+ *   - the Four-Over-Six block scale search over targets 6 and 4 (DeepRead
+ *     page, Method > 训练基础设施, adaptive block scaling);
+ *   - sliding-window self-attention with a global sink A_g and a shot sink
+ *     A_s over K_eff(t) = A_g u A_s u KV[t-W, t), overlapping tokens counted
+ *     once, A_s tracked by two pointers and re-bound on a prompt switch
+ *     (DeepRead page, Method > 算法层设计, Multi-Shot Attention Sink).
+ *
+ * Conventions for every entry point:
+ *   - "device" pointers are CUDA device memory owned by the CALLER (for
+ *     example torch tensors passed by data_ptr()).  The library never
+ *     allocates or frees device memory and never synchronizes a stream,
+ *     except nvfp4kv_workspace_status(), which synchronizes its stream.
+ *   - Work is enqueued on the caller's stream and runs asynchronously.
+ *     Argument errors are reported synchronously, before anything is
+ *     enqueued.  Launch failures map to NVFP4KV_ERR_CUDA.  Errors found by a
+ *     kernel while running (a bounded wait that gave up) are recorded in the
+ *     workspace's status word and read with nvfp4kv_workspace_status().
+ *   - bf16 tensors are IEEE bfloat16 bit patterns, token-major [T][H][d]
+ *     (row-major, d fastest), as a video DiT lays out K, V and Q.
+ *   - The CUDA kernels support head dimension d = 128 only
+ *     (NVFP4KV_ERR_UNSUPPORTED otherwise).  Tensor pointers must be 16-byte
+ *     aligned (NVFP4KV_ERR_ALIGNMENT).
+ *   - One workspace (and one cache) per stream: calls that share one and
+ *     overlap on the GPU race.
+ *
+ * Storage of one quantized chunk (the "rearranged, then quantized" cache of
+ * the researchpapers.dev page, 推理: W4A4 加流式 VAE), head-major:
+ *   k_codes, v_codes : uint8 [H][T_c][d/2]  two E2M1 codes per byte, element
+ *                      2j in the low nibble of byte j (sign = bit 3)
+ *   k_scales, v_scales: uint8 [H][T_c][d/16] E4M3 (fn) block scales, one per
+ *                      16 consecutive channels
+ *   k_mean           : float [H][d]   K-smoothing mean (added back on decode)
+ *   tensor_scales    : float [2]      s_K, s_V (FP32 tensor scales)
+ * Codes + block scales take (9/8)*T_c*H*d bytes against 4*T_c*H*d for bf16
+ * K and V (DeepRead page, Method > 推理基础设施).
+ */
+#ifndef NVFP4KV_H
+#define NVFP4KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* nvfp4kv_stream_t;
+
+typedef enum {
+    NVFP4KV_OK = 0,
+    NVFP4KV_ERR_INVALID_ARG = 1,     /* NULL pointer, negative or zero size, ... */
+    NVFP4KV_ERR_ALIGNMENT = 2,       /* a tensor pointer not 16-byte aligned */
+    NVFP4KV_ERR_UNSUPPORTED = 3,     /* d != 128, or no sm_100 device */
+    NVFP4KV_ERR_CAPACITY = 4,        /* too many chunks in a key set, layer out of range */
+    NVFP4KV_ERR_EMPTY_KEYSET = 5,    /* attention with no key chunk */
+    NVFP4KV_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed */
+    NVFP4KV_ERR_DEVICE_TIMEOUT = 7   /* a kernel's bounded wait gave up */
+} nvfp4kv_status;
+
+/* Device pointers to one quantized chunk (layouts above). */
+typedef struct {
+    uint8_t* k_codes;
+    uint8_t* k_scales;
+    uint8_t* v_codes;
+    uint8_t* v_scales;
+    float* k_mean;
+    float* tensor_scales;
+} nvfp4kv_chunk_view;
+
+/* Largest number of chunks one attention call can read. */
+#define NVFP4KV_MAX_KEY_CHUNKS 32
+
+/* ------------------------------------------------------------------ sizes */
+
+/* Bytes of one chunk buffer as carved by nvfp4kv_chunk_view_init: the
+ * (9/8)*T_c*H*d payload, the mean, the two tensor scales, each part padded to
+ * 256 bytes.  Returns 0 for invalid sizes. */
+size_t nvfp4kv_chunk_bytes(int T_c, int H, int d);
+
+/* Fill *out with the part pointers of a chunk buffer at `base` (device,
+ * 256-byte aligned, nvfp4kv_chunk_bytes() long).  No device access. */
+nvfp4kv_status nvfp4kv_chunk_view_init(void* base, int T_c, int H, int d,
+                                       nvfp4kv_chunk_view* out);
+
+/* Bytes of the scratch workspace the quantizer and the attention need for
+ * chunks of this shape (partial sums of the K-smoothing mean, per-block
+ * maxima, the grid barrier and the status word). */
+size_t nvfp4kv_workspace_bytes(int T_c, int H, int d);
+
+/* Zero the workspace's control words (status, barrier) on `stream`.  Call it
+ * once after allocating a workspace, and again after a call reported
+ * NVFP4KV_ERR_DEVICE_TIMEOUT. */
+nvfp4kv_status nvfp4kv_workspace_init(void* ws, size_t ws_bytes, nvfp4kv_stream_t stream);
+
+/* Synchronize `stream`, read the workspace's status word (OK or
+ * NVFP4KV_ERR_DEVICE_TIMEOUT) and clear it. */
+nvfp4kv_status nvfp4kv_workspace_status(void* ws, nvfp4kv_stream_t stream);
+
+/* ------------------------------------------------------------------ quantizer */
+
+/*
+ * Quantize one frame-chunk's K and V ([T_c][H][d] bf16, device) into `out`
+ * (DeepRead page, Method > 推理基础设施: chunk-level quantization,
+ * K-smoothing, NVFP4 micro-blocks; Four-Over-Six per block, Method >
+ * 训练基础设施).  Steps, per tensor:
+ *   K only: mean[h][c] over the chunk's tokens (fp32: sums of 64-token
+ *           segments, then the sum of the segments, then / T_c), and
+ *           X = K - mean; for V, X = V.
+ *   s = max|X| / (6*448)  (1 if the tensor is all zero).
+ *   each block of 16 channels: encode with its max mapped to 6 and to 4
+ *   (E4M3 block scale RNE/saturating, E2M1 codes RNE ties-to-even), keep the
+ *   4-encoding only if its squared error is strictly lower.
+ * Results are bit-identical to the reference definition above.
+ * ws: device workspace of nvfp4kv_workspace_bytes(T_c, H, d), initialized
+ * once by nvfp4kv_workspace_init.  K, V and the outputs must not overlap.
+ */
+nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int H, int d,
+                                      const nvfp4kv_chunk_view* out, void* ws,
+                                      nvfp4kv_stream_t stream);
+
+/*
+ * De-quantize a chunk back to [T_c][H][d] (device): x = decode(q) *
+ * (decode(scale) * s), plus mean for K, each step one fp32 operation.
+ * out_dtype 0 = float32 output, 1 = bf16 (the fp32 value rounded to nearest
+ * even).  K_out or V_out may be NULL to skip that tensor.
+ */
+nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, int d,
+                                  void* K_out, void* V_out, int out_dtype,
+                                  nvfp4kv_stream_t stream);
+
+/* ------------------------------------------------------------------ attention */
+
+/*
+ * O = softmax(scale * Q K_hat^T) V_hat over every key of the listed chunks
+ * (in any order; the caller passes the de-duplicated key set), with K_hat
+ * and V_hat the de-quantized cache, non-causal inside a chunk (DeepRead page,
+ * Method > 算法层设计; fused de-quantization, Method > 推理基础设施).
+ *   chunks: host array of n_chunks (1..NVFP4KV_MAX_KEY_CHUNKS) views, each of
+ *           T_c tokens, H heads, d = 128.
+ *   Q, O:   [T_q][H][d] bf16, device; O is written, Q is read.
+ *   softmax_scale: <= 0 selects 1/sqrt(d).
+ *   ws:     workspace as for the quantizer (status word only).
+ * Softmax statistics are fp32; the products run on the tensor cores in bf16
+ * with the de-quantized values exact in bf16; the result is rounded to bf16.
+ */
+nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
+                                 int T_c, int H, int d, const void* Q, int T_q,
+                                 void* O, float softmax_scale, void* ws,
+                                 nvfp4kv_stream_t stream);
+
+/* ------------------------------------------------------------------ cache */
+
+/* Cache shape.  Sinks and window count whole chunks (a chunk = F_c frames of
+ * T_c tokens, DeepRead page, Method > 推理基础设施): S_g global-sink chunks
+ * [0, S_g), S_s shot-sink chunks from the current shot's first chunk, and the
+ * W newest chunks including the one just appended. */
+typedef struct {
+    int layers;
+    int H;
+    int d;
+    int T_c;
+    int S_g;
+    int S_s;
+    int W;
+} kvcache_config;
+
+typedef struct kvcache kvcache;   /* host object; opaque */
+
+/* Slots per layer (S_g + S_s + W, at least 1) times layers times
+ * nvfp4kv_chunk_bytes(T_c, H, d). */
+size_t kvcache_pool_bytes(const kvcache_config* cfg);
+
+/*
+ * Create a cache over caller-owned device memory: `pool` of
+ * kvcache_pool_bytes() (256-byte aligned) and `ws` of
+ * nvfp4kv_workspace_bytes(T_c, H, d).  No device access: the first
+ * kvcache_append zeroes the workspace's control words on its own stream.  The
+ * shot sink starts at chunk 0.  *out is a host object released with
+ * kvcache_destroy.
+ */
+nvfp4kv_status kvcache_create(const kvcache_config* cfg, void* pool, void* ws, kvcache** out);
+void kvcache_destroy(kvcache* cache);
+
+/*
+ * Append the next chunk of `layer`: chunk id n = number of chunks appended to
+ * this layer so far.  Frees the slots of chunks that leave A_g u A_s u the
+ * window, then quantizes K and V ([T_c][H][d] bf16, device) into a free slot
+ * in place, on `stream`.  A chunk that no future attention can read (W = 0
+ * and not a sink chunk) is counted but not stored.
+ */
+nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const void* V,
+                              nvfp4kv_stream_t stream);
+
+/*
+ * Prompt switch p_k -> p_k' (DeepRead page, Method > 算法层设计): the shot
+ * sink moves to [first_chunk_of_shot, first_chunk_of_shot + S_s) for every
+ * layer; the global sink and the history are kept.  Call it before appending
+ * that chunk.  Host bookkeeping only (two pointers, no device memory).
+ * NVFP4KV_ERR_INVALID_ARG (nothing changed) if a chunk of the new sink was
+ * appended to some layer already and is no longer stored there.
+ */
+nvfp4kv_status kvcache_rebind_shot_sink(kvcache* cache, int64_t first_chunk_of_shot);
+
+/* The sorted, de-duplicated chunk ids `layer` attends now, written to ids
+ * (room for S_g + S_s + W entries); *count receives their number. */
+nvfp4kv_status kvcache_keyset(const kvcache* cache, int layer, int64_t* ids, int* count);
+
+/* Chunks appended to `layer` so far. */
+nvfp4kv_status kvcache_num_chunks(const kvcache* cache, int layer, int64_t* n);
+
+/* Device views of a stored chunk (NVFP4KV_ERR_INVALID_ARG if not stored). */
+nvfp4kv_status kvcache_chunk_view(const kvcache* cache, int layer, int64_t chunk,
+                                  nvfp4kv_chunk_view* out);
+
+/*
+ * Bookkeeping half of kvcache_append without the quantization: frees slots
+ * leaving the key set, claims one for the next chunk and returns its view in
+ * *out (out->k_codes == NULL when the chunk is not stored).  For callers that
+ * fill the slot themselves, and for host-side tests.
+ */
+nvfp4kv_status kvcache_advance(kvcache* cache, int layer, nvfp4kv_chunk_view* out);
+
+/*
+ * Sink-window attention of `layer`'s queries Q [T_q][H][d] (bf16, device)
+ * over its current key set, written to O [T_q][H][d] (bf16, device): the
+ * key set of kvcache_keyset() passed to nvfp4kv_attention().
+ * NVFP4KV_ERR_EMPTY_KEYSET if no chunk is attended.
+ */
+nvfp4kv_status sink_window_attention(const kvcache* cache, int layer, const void* Q, int T_q,
+                                     void* O, float softmax_scale, nvfp4kv_stream_t stream);
+
+/* The cache's workspace status (see nvfp4kv_workspace_status). */
+nvfp4kv_status kvcache_check_status(kvcache* cache, nvfp4kv_stream_t stream);
+
+/* ------------------------------------------------------------------ checks */
+
+/*
+ * Element-wise use of the GPU's own format conversions, exported so that
+ * tests can compare them with a reference on every input they choose:
+ * op 0: E2M1 code of each fp32 input (one code per output byte),
+ * op 1: E4M3 byte of each fp32 input, op 2: fp32 value of each E2M1 code,
+ * op 3: fp32 value of each E4M3 byte, op 4: the fp32 quotient x/D that the
+ * quantizer forms for a pair (in[2i] = x, in[2i+1] = D > 0).
+ * in/out are device arrays of n elements (op 4: n quotients from 2n inputs).
+ */
+nvfp4kv_status nvfp4kv_check_formats(int op, const void* in, void* out, size_t n,
+                                     nvfp4kv_stream_t stream);
+
+/* Library version string. */
+const char* nvfp4kv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4KV_H */

@@ -1,0 +1,307 @@
+"""Python binding of libnvfp4kv (NVFP4 KV cache + multi-shot sink-window
+attention for B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory and streams.  The binding fails
+loudly when the compiled library is missing; there is no fallback path.
+
+The names mirror the C ABI in include/nvfp4kv.h.
+"""
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4kv.so")
+
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_EMPTY_KEYSET, \
+    ERR_CUDA, ERR_DEVICE_TIMEOUT = range(8)
+STATUS_NAMES = ["OK", "ERR_INVALID_ARG", "ERR_ALIGNMENT", "ERR_UNSUPPORTED", "ERR_CAPACITY",
+                "ERR_EMPTY_KEYSET", "ERR_CUDA", "ERR_DEVICE_TIMEOUT"]
+MAX_KEY_CHUNKS = 32
+HEAD_DIM = 128
+
+_lib = None
+
+
+class NvFp4KvError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = status
+        name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else str(status)
+        super().__init__(f"{where}: {name}")
+
+
+class ChunkView(ctypes.Structure):
+    """nvfp4kv_chunk_view: device pointers to one quantized chunk."""
+    _fields_ = [("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+                ("v_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("k_mean", ctypes.c_void_p), ("tensor_scales", ctypes.c_void_p)]
+
+
+class KVCacheConfig(ctypes.Structure):
+    _fields_ = [("layers", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("T_c", ctypes.c_int), ("S_g", ctypes.c_int), ("S_s", ctypes.c_int),
+                ("W", ctypes.c_int)]
+
+
+def load():
+    """Load libnvfp4kv.so (built by sink_window_video_b200/build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python sink_window_video_b200/build.py` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz, f32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                             ctypes.c_float)
+    st = ctypes.c_int
+    cv = ctypes.POINTER(ChunkView)
+    cfgp = ctypes.POINTER(KVCacheConfig)
+    sigs = {
+        "nvfp4kv_chunk_bytes": (sz, [i32, i32, i32]),
+        "nvfp4kv_chunk_view_init": (st, [vp, i32, i32, i32, cv]),
+        "nvfp4kv_workspace_bytes": (sz, [i32, i32, i32]),
+        "nvfp4kv_workspace_init": (st, [vp, sz, vp]),
+        "nvfp4kv_workspace_status": (st, [vp, vp]),
+        "nvfp4kv_quantize_chunk": (st, [vp, vp, i32, i32, i32, cv, vp, vp]),
+        "nvfp4kv_dequantize": (st, [cv, i32, i32, i32, vp, vp, i32, vp]),
+        "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, f32, vp, vp]),
+        "kvcache_pool_bytes": (sz, [cfgp]),
+        "kvcache_create": (st, [cfgp, vp, vp, ctypes.POINTER(vp)]),
+        "kvcache_destroy": (None, [vp]),
+        "kvcache_append": (st, [vp, i32, vp, vp, vp]),
+        "kvcache_rebind_shot_sink": (st, [vp, i64]),
+        "kvcache_keyset": (st, [vp, i32, ctypes.POINTER(i64), ctypes.POINTER(i32)]),
+        "kvcache_num_chunks": (st, [vp, i32, ctypes.POINTER(i64)]),
+        "kvcache_chunk_view": (st, [vp, i32, i64, cv]),
+        "kvcache_advance": (st, [vp, i32, cv]),
+        "sink_window_attention": (st, [vp, i32, vp, i32, vp, f32, vp]),
+        "kvcache_check_status": (st, [vp, vp]),
+        "nvfp4kv_check_formats": (st, [i32, vp, vp, sz, vp]),
+        "nvfp4kv_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status, where):
+    if status != OK:
+        raise NvFp4KvError(status, where)
+
+
+def _ptr(x):
+    """Device address of a torch tensor (or an int / None)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def version() -> str:
+    return load().nvfp4kv_version().decode()
+
+
+# ------------------------------------------------------------------ sizes
+
+def chunk_bytes(T_c, H, d=HEAD_DIM) -> int:
+    return int(load().nvfp4kv_chunk_bytes(T_c, H, d))
+
+
+def workspace_bytes(T_c, H, d=HEAD_DIM) -> int:
+    return int(load().nvfp4kv_workspace_bytes(T_c, H, d))
+
+
+def chunk_view_init(base, T_c, H, d=HEAD_DIM) -> ChunkView:
+    v = ChunkView()
+    _check(load().nvfp4kv_chunk_view_init(_ptr(base), T_c, H, d, ctypes.byref(v)),
+           "nvfp4kv_chunk_view_init")
+    return v
+
+
+def workspace_init(ws, stream=None):
+    _check(load().nvfp4kv_workspace_init(_ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "nvfp4kv_workspace_init")
+
+
+def workspace_status(ws, stream=None) -> int:
+    """Synchronize and return the workspace status code (OK or ERR_DEVICE_TIMEOUT)."""
+    return int(load().nvfp4kv_workspace_status(_ptr(ws), _stream(stream)))
+
+
+# ------------------------------------------------------------------ device buffers
+
+class ChunkBuffer:
+    """One quantized chunk in a torch uint8 device buffer, with torch views of
+    its parts (codes [H, T, d/2], scales [H, T, d/16], k_mean [H, d],
+    tensor_scales [2])."""
+
+    def __init__(self, T_c, H, d=HEAD_DIM, device="cuda", buf=None):
+        import torch
+        self.T_c, self.H, self.d = T_c, H, d
+        n = chunk_bytes(T_c, H, d)
+        self.buf = buf if buf is not None else torch.zeros(n + 256, dtype=torch.uint8,
+                                                           device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.base = self.buf[off:off + n]
+        self.view = chunk_view_init(self.base, T_c, H, d)
+        b0 = self.base.data_ptr()
+
+        def part(ptr, nbytes):
+            return self.base[ptr - b0: ptr - b0 + nbytes]
+        nn = T_c * H * d
+        self.k_codes = part(self.view.k_codes, nn // 2).view(H, T_c, d // 2)
+        self.v_codes = part(self.view.v_codes, nn // 2).view(H, T_c, d // 2)
+        self.k_scales = part(self.view.k_scales, nn // 16).view(H, T_c, d // 16)
+        self.v_scales = part(self.view.v_scales, nn // 16).view(H, T_c, d // 16)
+        self.k_mean = part(self.view.k_mean, H * d * 4).view(torch.float32).view(H, d)
+        self.tensor_scales = part(self.view.tensor_scales, 8).view(torch.float32)
+
+    def to_host(self):
+        """dict of numpy arrays in the layout the oracle uses."""
+        return dict(k_codes=self.k_codes.cpu().numpy(), k_scales=self.k_scales.cpu().numpy(),
+                    v_codes=self.v_codes.cpu().numpy(), v_scales=self.v_scales.cpu().numpy(),
+                    k_mean=self.k_mean.cpu().numpy(),
+                    s_k=float(self.tensor_scales[0].item()),
+                    s_v=float(self.tensor_scales[1].item()), T=self.T_c)
+
+
+def new_workspace(T_c, H, d=HEAD_DIM, device="cuda", stream=None):
+    """A zeroed torch uint8 workspace (256-byte aligned) for chunks of this shape."""
+    import torch
+    n = workspace_bytes(T_c, H, d)
+    ws = torch.zeros(n, dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    workspace_init(ws, stream)
+    return ws
+
+
+# ------------------------------------------------------------------ quantizer
+
+def quantize_chunk(K, V, out: ChunkBuffer, ws, stream=None):
+    """K, V: bf16 [T_c, H, d] device tensors -> out (a ChunkBuffer)."""
+    T, H, d = K.shape
+    _check(load().nvfp4kv_quantize_chunk(_ptr(K), _ptr(V), T, H, d, ctypes.byref(out.view),
+                                         _ptr(ws), _stream(stream)), "nvfp4kv_quantize_chunk")
+
+
+def dequantize(chunk: ChunkBuffer, K_out=None, V_out=None, stream=None):
+    """Write de-quantized [T_c, H, d] K and/or V (float32 or bf16 tensors)."""
+    import torch
+    t = K_out if K_out is not None else V_out
+    dtype = 1 if t.dtype == torch.bfloat16 else 0
+    _check(load().nvfp4kv_dequantize(ctypes.byref(chunk.view), chunk.T_c, chunk.H, chunk.d,
+                                     _ptr(K_out), _ptr(V_out), dtype, _stream(stream)),
+           "nvfp4kv_dequantize")
+
+
+def attention(chunks, Q, O, ws, softmax_scale=0.0, stream=None):
+    """O = softmax(scale Q K^T) V over the listed chunks (ChunkBuffer or ChunkView)."""
+    views = [c.view if hasattr(c, "view") else c for c in chunks]
+    arr = (ChunkView * max(1, len(views)))(*views)
+    first = chunks[0] if chunks else None
+    T_c = first.T_c if hasattr(first, "T_c") else 0
+    T_q, H, d = Q.shape
+    _check(load().nvfp4kv_attention(arr, len(views), T_c, H, d, _ptr(Q), T_q, _ptr(O),
+                                    float(softmax_scale), _ptr(ws), _stream(stream)),
+           "nvfp4kv_attention")
+
+
+def check_formats(op, inp, out, n=None, stream=None):
+    n = inp.numel() if n is None else n
+    _check(load().nvfp4kv_check_formats(op, _ptr(inp), _ptr(out), n, _stream(stream)),
+           "nvfp4kv_check_formats")
+
+
+# ------------------------------------------------------------------ cache
+
+class KVCache:
+    """kvcache over torch-allocated device memory (pool + workspace)."""
+
+    def __init__(self, layers, H, T_c, S_g, S_s, W, d=HEAD_DIM, device="cuda", pool=None,
+                 ws=None):
+        import torch
+        L = load()
+        self.cfg = KVCacheConfig(layers, H, d, T_c, S_g, S_s, W)
+        self.T_c, self.H, self.d, self.layers = T_c, H, d, layers
+        n = int(L.kvcache_pool_bytes(ctypes.byref(self.cfg)))
+        if n == 0:
+            raise NvFp4KvError(ERR_INVALID_ARG, "kvcache_pool_bytes")
+        self.pool = pool if pool is not None else torch.empty(n, dtype=torch.uint8, device=device)
+        self.ws = ws if ws is not None else torch.zeros(workspace_bytes(T_c, H, d),
+                                                        dtype=torch.uint8, device=device)
+        self._h = ctypes.c_void_p()
+        _check(L.kvcache_create(ctypes.byref(self.cfg), _ptr(self.pool), _ptr(self.ws),
+                                ctypes.byref(self._h)), "kvcache_create")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.kvcache_destroy(h)
+            self._h = None
+
+    def append(self, layer, K, V, stream=None):
+        _check(load().kvcache_append(self._h, layer, _ptr(K), _ptr(V), _stream(stream)),
+               "kvcache_append")
+
+    def advance(self, layer):
+        v = ChunkView()
+        _check(load().kvcache_advance(self._h, layer, ctypes.byref(v)), "kvcache_advance")
+        return v
+
+    def rebind_shot_sink(self, first_chunk_of_shot):
+        _check(load().kvcache_rebind_shot_sink(self._h, int(first_chunk_of_shot)),
+               "kvcache_rebind_shot_sink")
+
+    def keyset(self, layer):
+        ids = (ctypes.c_int64 * MAX_KEY_CHUNKS)()
+        cnt = ctypes.c_int()
+        _check(load().kvcache_keyset(self._h, layer, ids, ctypes.byref(cnt)), "kvcache_keyset")
+        return [int(ids[i]) for i in range(cnt.value)]
+
+    def num_chunks(self, layer):
+        n = ctypes.c_int64()
+        _check(load().kvcache_num_chunks(self._h, layer, ctypes.byref(n)), "kvcache_num_chunks")
+        return int(n.value)
+
+    def chunk_view(self, layer, chunk) -> ChunkView:
+        v = ChunkView()
+        _check(load().kvcache_chunk_view(self._h, layer, int(chunk), ctypes.byref(v)),
+               "kvcache_chunk_view")
+        return v
+
+    def chunk(self, layer, chunk) -> ChunkBuffer:
+        """Torch views of a stored chunk (device memory of the pool)."""
+        v = self.chunk_view(layer, chunk)
+        off = v.k_codes - self.pool.data_ptr()
+        buf = ChunkBuffer.__new__(ChunkBuffer)
+        n = chunk_bytes(self.T_c, self.H, self.d)
+        ChunkBuffer.__init__(buf, self.T_c, self.H, self.d, buf=self.pool[off:off + n])
+        return buf
+
+    def attention(self, layer, Q, O, softmax_scale=0.0, stream=None):
+        T_q = Q.shape[0]
+        _check(load().sink_window_attention(self._h, layer, _ptr(Q), T_q, _ptr(O),
+                                            float(softmax_scale), _stream(stream)),
+               "sink_window_attention")
+
+    def check_status(self, stream=None) -> int:
+        return int(load().kvcache_check_status(self._h, _stream(stream)))
+
+
+def default_scale(d=HEAD_DIM):
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,58 @@
+// kernels.h -- host-side entry points of the CUDA kernels (internal to the
+// library; the public C ABI is include/nvfp4kv.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "nvfp4kv.h"
+
+namespace nvfp4kv {
+
+constexpr int kMaxGrid = 4096;       // room for per-CTA partials in the workspace
+constexpr int kHeadDimSupported = 128;   // head dimension d the kernels support
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace layout for chunks of T tokens and H heads (d = 128):
+//   [0, 256)  Control (status word, grid barrier)
+//   psum      float    [nseg][H*d]  per-segment column sums of K
+//   pmin/pmax bf16     [nseg][H*d]  per-segment column min / max of K
+//   kpart     float    [kMaxGrid]   per-CTA max |K - mean|
+//   vpart     float    [kMaxGrid]   per-CTA max |V|
+struct WsLayout {
+    size_t psum, pmin, pmax, kpart, vpart, total;
+};
+
+inline WsLayout ws_layout(int T, int H) {
+    size_t HD = (size_t)H * 128;
+    size_t nseg = ((size_t)T + 63) / 64;
+    WsLayout L;
+    size_t off = 256;
+    L.psum = off;  off += align256(nseg * HD * 4);
+    L.pmin = off;  off += align256(nseg * HD * 2);
+    L.pmax = off;  off += align256(nseg * HD * 2);
+    L.kpart = off; off += align256(kMaxGrid * 4);
+    L.vpart = off; off += align256(kMaxGrid * 4);
+    L.total = off;
+    return L;
+}
+
+nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
+                               const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream);
+
+nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, void* K_out,
+                                 void* V_out, int out_dtype, cudaStream_t stream);
+
+nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,
+                                    cudaStream_t stream);
+
+nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                    int H, const void* Q, int T_q, void* O, float softmax_scale,
+                                    cudaStream_t stream);
+
+nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                int H, const void* Q, int T_q, void* O, float softmax_scale,
+                                void* ws, cudaStream_t stream);
+
+}  // namespace nvfp4kv

@@ -1,0 +1,171 @@
+"""The C-ABI library on the host (no GPU work): it loads, exports every
+symbol include/nvfp4kv.h declares, lays chunks out in (9/8)*T*H*d payload
+bytes, rejects bad arguments before touching a device, and its cache
+bookkeeping (slot pool, eviction, shot-sink rebinding) keeps exactly the key
+set of the oracle.  Pointers passed here are never dereferenced: every call
+either does host bookkeeping only or fails validation first."""
+import ctypes
+import os
+import random
+import re
+import subprocess
+import sys
+
+import pytest
+
+import sink_window_video_b200 as swv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4kv.h")
+FAKE = 0x7F0000000000      # 256-byte aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(swv.LIB_PATH):
+        from sink_window_video_b200 import build
+        build.build()
+    return swv.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return sorted({n for n in names if n not in ("if", "defined")})
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 20
+    out = subprocess.run(["nm", "-D", "--defined-only", swv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+
+
+def test_chunk_layout_holds_the_payload(L):
+    for T, H in [(7040, 24), (32, 2), (48, 3)]:
+        n = T * H * 128
+        cb = swv.chunk_bytes(T, H)
+        assert cb % 256 == 0 and cb >= n * 9 // 8 + H * 128 * 4 + 8
+        assert cb - (n * 9 // 8 + H * 128 * 4 + 8) < 6 * 256
+        v = swv.chunk_view_init(FAKE, T, H)
+        parts = sorted([(v.k_codes, n // 2), (v.v_codes, n // 2), (v.k_scales, n // 16),
+                        (v.v_scales, n // 16), (v.k_mean, H * 128 * 4), (v.tensor_scales, 8)])
+        for (a, na), (b, _) in zip(parts, parts[1:]):
+            assert a + na <= b                       # no overlap
+        assert parts[-1][0] + parts[-1][1] <= FAKE + cb
+        assert all(p % 16 == 0 for p, _ in parts)
+    assert swv.chunk_bytes(0, 2) == 0 and swv.chunk_bytes(32, 2, 100) == 0
+
+
+def test_rejects_bad_arguments_without_device_work(L):
+    cv = swv.ChunkView(FAKE, FAKE + 4096, FAKE + 8192, FAKE + 12288, FAKE + 16384, FAKE + 20480)
+    q = L.nvfp4kv_quantize_chunk
+    assert q(None, FAKE, 32, 2, 128, ctypes.byref(cv), FAKE, None) == swv.ERR_INVALID_ARG
+    assert q(FAKE, FAKE, 0, 2, 128, ctypes.byref(cv), FAKE, None) == swv.ERR_INVALID_ARG
+    assert q(FAKE, FAKE, 32, 2, 64, ctypes.byref(cv), FAKE, None) == swv.ERR_UNSUPPORTED
+    assert q(FAKE + 8, FAKE, 32, 2, 128, ctypes.byref(cv), FAKE, None) == swv.ERR_ALIGNMENT
+    assert q(FAKE, FAKE, 32, 2, 128, ctypes.byref(cv), FAKE + 16, None) == swv.ERR_ALIGNMENT
+    a = L.nvfp4kv_attention
+    arr = (swv.ChunkView * 1)(cv)
+    assert a(arr, 0, 32, 2, 128, FAKE, 32, FAKE, 0.0, FAKE, None) == swv.ERR_EMPTY_KEYSET
+    assert a(arr, 33, 32, 2, 128, FAKE, 32, FAKE, 0.0, FAKE, None) == swv.ERR_CAPACITY
+    assert a(arr, 1, 32, 2, 128, FAKE + 4, 32, FAKE, 0.0, FAKE, None) == swv.ERR_ALIGNMENT
+    assert a(arr, 1, 32, 2, 96, FAKE, 32, FAKE, 0.0, FAKE, None) == swv.ERR_UNSUPPORTED
+    assert L.nvfp4kv_check_formats(9, FAKE, FAKE, 1, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_workspace_init(None, 256, None) == swv.ERR_INVALID_ARG
+
+
+def _cache(L, layers, S_g, S_s, W, T=32, H=2):
+    cfg = swv.KVCacheConfig(layers, H, 128, T, S_g, S_s, W)
+    h = ctypes.c_void_p()
+    assert L.kvcache_create(ctypes.byref(cfg), FAKE, FAKE, ctypes.byref(h)) == swv.OK
+    return h, cfg
+
+
+def _keyset(L, h, layer):
+    ids = (ctypes.c_int64 * 64)()
+    n = ctypes.c_int()
+    assert L.kvcache_keyset(h, layer, ids, ctypes.byref(n)) == swv.OK
+    return [ids[i] for i in range(n.value)]
+
+
+def test_cache_bookkeeping_matches_oracle_keyset(L, orc):
+    rng = random.Random(3)
+    for trial in range(60):
+        S_g, S_s, W = rng.randint(0, 3), rng.randint(0, 3), rng.randint(0, 5)
+        if S_g + S_s + W == 0:
+            W = 1
+        layers = rng.randint(1, 3)
+        h, cfg = _cache(L, layers, S_g, S_s, W)
+        slots = S_g + S_s + W
+        cb = swv.chunk_bytes(32, 2)
+        pool_end = FAKE + swv.load().kvcache_pool_bytes(ctypes.byref(cfg))
+        s_begin = 0
+        n = [0] * layers
+        for step in range(rng.randint(5, 40)):
+            if rng.random() < 0.15:
+                # the next shot starts at or after the newest chunk of every layer
+                s_begin = max(n) + rng.randint(0, 2)
+                assert L.kvcache_rebind_shot_sink(h, s_begin) == swv.OK
+            if rng.random() < 0.1 and S_s > 0:
+                # a shot sink on past chunks is accepted only if every layer that
+                # appended them still stores them; otherwise refused, state kept
+                stale = rng.randint(0, max(n))
+                cv = swv.ChunkView()
+                ok = all(L.kvcache_chunk_view(h, ly, c, ctypes.byref(cv)) == swv.OK
+                         for ly in range(layers)
+                         for c in range(stale, min(stale + S_s, n[ly])))
+                st = L.kvcache_rebind_shot_sink(h, stale)
+                assert st == (swv.OK if ok else swv.ERR_INVALID_ARG)
+                if ok:
+                    s_begin = stale
+            layer = rng.randrange(layers)
+            v = swv.ChunkView()
+            assert L.kvcache_advance(h, layer, ctypes.byref(v)) == swv.OK
+            n[layer] += 1
+            ids = _keyset(L, h, layer)
+            assert ids == orc.keyset(n[layer], S_g, S_s, W, s_begin)
+            stored = []
+            for c in range(n[layer]):
+                cv = swv.ChunkView()
+                st = L.kvcache_chunk_view(h, layer, c, ctypes.byref(cv))
+                if st == swv.OK:
+                    stored.append((c, cv.k_codes))
+            # every attended chunk is stored; nothing else is kept past its use
+            live_next = set(orc.keyset(n[layer] + 1, S_g, S_s, W, s_begin)) | set(ids)
+            assert set(ids) <= {c for c, _ in stored}
+            assert {c for c, _ in stored} <= live_next
+            assert len(stored) <= slots
+            addrs = [a for _, a in stored]
+            assert len(set(addrs)) == len(addrs)
+            assert all(FAKE <= a < pool_end for a in addrs)
+            assert all((a - FAKE) % cb == 0 for a in addrs)
+            cnt = ctypes.c_int64()
+            assert L.kvcache_num_chunks(h, layer, ctypes.byref(cnt)) == swv.OK
+            assert cnt.value == n[layer]
+        L.kvcache_destroy(h)
+
+
+def test_cache_rejects_bad_layers_and_sizes(L):
+    h, _ = _cache(L, 2, 1, 1, 2)
+    v = swv.ChunkView()
+    assert L.kvcache_advance(h, 2, ctypes.byref(v)) == swv.ERR_CAPACITY
+    assert L.kvcache_advance(h, -1, ctypes.byref(v)) == swv.ERR_CAPACITY
+    assert L.kvcache_rebind_shot_sink(h, -3) == swv.ERR_INVALID_ARG
+    # no chunk yet: nothing to attend, reported before any launch
+    assert L.sink_window_attention(h, 0, FAKE, 32, FAKE, 0.0, None) == swv.ERR_EMPTY_KEYSET
+    L.kvcache_destroy(h)
+    cfg = swv.KVCacheConfig(1, 2, 128, 32, 20, 10, 10)
+    hh = ctypes.c_void_p()
+    assert L.kvcache_create(ctypes.byref(cfg), FAKE, FAKE, ctypes.byref(hh)) == swv.ERR_CAPACITY
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    code = ("import sink_window_video_b200 as s; s.LIB_PATH = '/nonexistent/libnvfp4kv.so'\n"
+            "try:\n    s.load()\nexcept ImportError as e:\n    print('LOUD', e)\n")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT)
+    assert "LOUD" in r.stdout

@@ -1,0 +1,142 @@
+"""GPU sink-window attention against the float64 oracle (relative L2 <= 1e-2,
+max-abs <= 2e-2), through the cache (kvcache_append / sink_window_attention)
+and through the explicit-list entry point (nvfp4kv_attention).  The oracle
+attends over chunks quantized by the oracle itself from the same inputs (the
+quantizers agree bit for bit, tested separately)."""
+import numpy as np
+import pytest
+
+import synth
+from gpu_util import assert_attention_close, dev_bf16, host_bf16_to_f64, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def _attend(lib, cache, layer, Q):
+    import torch
+    O = torch.empty((Q.shape[0],) + Q.shape[1:], dtype=torch.bfloat16, device="cuda")
+    cache.attention(layer, dev_bf16(Q), O)
+    torch.cuda.synchronize()
+    assert cache.check_status() == lib.OK
+    return host_bf16_to_f64(O)
+
+
+def test_tiny_config_rollout(lib, orc):
+    c = synth.TINY
+    cache = lib.KVCache(1, c["H"], c["T_c"], c["S_g"], c["S_s"], c["W"])
+    qs = []
+    for n in range(c["chunks"]):
+        K, V, Q = synth.tiny_chunk(n)
+        cache.append(0, dev_bf16(K), dev_bf16(V))
+        qs.append(orc.quantize_chunk(K, V))
+        ids = cache.keyset(0)
+        assert ids == orc.keyset(n + 1, c["S_g"], c["S_s"], c["W"], 0)
+        out = _attend(lib, cache, 0, Q)
+        ref = orc.attention_f64([qs[i] for i in ids], Q)
+        assert_attention_close(out, ref, f"tiny chunk {n}")
+
+
+def test_one_layer_attention_full_size(lib, orc):
+    """One layer at the 5B DiT shape: Q [7040, 24, 128] over the global sink {0},
+    the shot sink {4} and the window {7, 8, 9}: 35,200 keys."""
+    c = synth.ATTN
+    cache = lib.KVCache(1, c["H"], c["T_c"], c["S_g"], c["S_s"], c["W"])
+    want_ids = [0, 4, 7, 8, 9]
+    qs = {}
+    for n in range(c["appended"]):
+        if n == c["shot_start"]:
+            cache.rebind_shot_sink(n)
+        K, V, Q = synth.layer_chunk(c, 0, n)
+        cache.append(0, dev_bf16(K), dev_bf16(V))
+        if n in want_ids:
+            qs[n] = orc.quantize_chunk(K, V)
+    assert cache.keyset(0) == want_ids
+    out = _attend(lib, cache, 0, Q)
+    rows = sample_rows(c["T_c"], n_random=24, seed=2)
+    ref = orc.attention_f64([qs[i] for i in want_ids], Q, rows=rows)
+    assert_attention_close(out[rows], ref, "one-layer attention")
+
+
+@pytest.mark.parametrize("T_c,T_q,H", [(48, 100, 2), (136, 136, 3), (200, 7, 2), (1, 5, 2),
+                                       (129, 257, 1)])
+def test_ragged_shapes(lib, orc, T_c, T_q, H):
+    import torch
+    n_chunks = 3
+    chunks, qs = [], []
+    ws = lib.new_workspace(T_c, H)
+    for i in range(n_chunks):
+        K = synth.k_with_offsets_bf16(50 + i, T_c, H, (T_c, H, 128))
+        V = synth.gaussian_bf16(50 + i, T_c, H, synth.T_V, (T_c, H, 128))
+        buf = lib.ChunkBuffer(T_c, H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), buf, ws)
+        chunks.append(buf)
+        qs.append(orc.quantize_chunk(K, V))
+    Q = synth.gaussian_bf16(60, T_c, H, synth.T_Q, (T_q, H, 128))
+    O = torch.empty((T_q, H, 128), dtype=torch.bfloat16, device="cuda")
+    lib.attention(chunks, dev_bf16(Q), O, ws)
+    torch.cuda.synchronize()
+    assert_attention_close(host_bf16_to_f64(O), orc.attention_f64(qs, Q), f"T_c={T_c} T_q={T_q}")
+
+
+def test_duplicated_list_counts_twice(lib, orc):
+    """The explicit-list entry point attends to exactly what it is given."""
+    import torch
+    T_c, H = 64, 2
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i in range(2):
+        K, V, _ = synth.tiny_chunk(i)
+        K, V = K[:T_c], V[:T_c]
+        b = lib.ChunkBuffer(K.shape[0], H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), b, ws)
+        bufs.append(b)
+        qs.append(orc.quantize_chunk(K, V))
+    _, _, Q = synth.tiny_chunk(3)
+    O = torch.empty(Q.shape, dtype=torch.bfloat16, device="cuda")
+    lib.attention([bufs[0], bufs[0], bufs[1]], dev_bf16(Q), O, ws)
+    torch.cuda.synchronize()
+    out = host_bf16_to_f64(O)
+    assert_attention_close(out, orc.attention_f64([qs[0], qs[0], qs[1]], Q), "duplicated")
+    uniq = orc.attention_f64([qs[0], qs[1]], Q)
+    assert np.abs(out - uniq).max() > 5e-2
+
+
+def test_window_zero_is_sink_only(lib, orc):
+    """W = 0: only the global and shot sinks are attended; other chunks are not
+    even stored."""
+    H, T_c = 2, 32
+    cache = lib.KVCache(1, H, T_c, S_g=1, S_s=1, W=0)
+    qs = {}
+    for n in range(5):
+        if n == 2:
+            cache.rebind_shot_sink(2)
+        K, V, Q = synth.tiny_chunk(n)
+        cache.append(0, dev_bf16(K), dev_bf16(V))
+        qs[n] = orc.quantize_chunk(K, V)
+    assert cache.keyset(0) == [0, 2]
+    out = _attend(lib, cache, 0, Q)
+    assert_attention_close(out, orc.attention_f64([qs[0], qs[2]], Q), "W=0")
+
+
+def test_overlapping_sinks_deduplicated(lib, orc):
+    H, T_c = 2, 32
+    cache = lib.KVCache(1, H, T_c, S_g=2, S_s=2, W=2)
+    qs = {}
+    for n in range(4):
+        K, V, Q = synth.tiny_chunk(n)
+        cache.append(0, dev_bf16(K), dev_bf16(V))
+        qs[n] = orc.quantize_chunk(K, V)
+    # A_g = {0,1}, A_s = {0,1} (shot 0), window = {2,3}
+    assert cache.keyset(0) == [0, 1, 2, 3]
+    out = _attend(lib, cache, 0, Q)
+    assert_attention_close(out, orc.attention_f64([qs[i] for i in range(4)], Q), "dedup")
+
+
+def test_empty_keyset_is_an_error(lib):
+    import torch
+    cache = lib.KVCache(1, 2, 32, S_g=1, S_s=1, W=1)
+    Q = torch.zeros((32, 2, 128), dtype=torch.bfloat16, device="cuda")
+    O = torch.empty_like(Q)
+    with pytest.raises(lib.NvFp4KvError) as e:
+        cache.attention(0, Q, O)
+    assert e.value.status == lib.ERR_EMPTY_KEYSET

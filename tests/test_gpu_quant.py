@@ -1,0 +1,114 @@
+"""GPU quantizer and de-quantizer against the oracle, bit for bit: FP4 codes,
+E4M3 scale bytes, the K-smoothing mean and both tensor scales, on the tiny
+configuration, on full-size quantize-only chunks (7040 x 24 x 128) and on
+ragged and degenerate shapes."""
+import numpy as np
+import pytest
+
+import synth
+from gpu_util import dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_quant(lib, K, V, ws=None):
+    import torch
+    T, H, d = K.shape
+    ws = lib.new_workspace(T, H, d) if ws is None else ws
+    out = lib.ChunkBuffer(T, H, d)
+    lib.quantize_chunk(dev_bf16(K), dev_bf16(V), out, ws)
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    return out, ws
+
+
+def _assert_same(gpu: dict, ref: dict, what=""):
+    for k in ("k_codes", "k_scales", "v_codes", "v_scales"):
+        a, b = gpu[k], ref[k]
+        if not np.array_equal(a, b):
+            idx = np.argwhere(a != b)
+            raise AssertionError(f"{what} {k}: {len(idx)} bytes differ, first at {idx[:4].tolist()}")
+    assert np.array_equal(gpu["k_mean"].view(np.uint32), ref["k_mean"].view(np.uint32)), \
+        f"{what} k_mean differs"
+    assert np.float32(gpu["s_k"]) == np.float32(ref["s_k"]), f"{what} s_K"
+    assert np.float32(gpu["s_v"]) == np.float32(ref["s_v"]), f"{what} s_V"
+
+
+def test_tiny_config_bit_exact(lib, orc):
+    ws = None
+    for c in range(synth.TINY["chunks"]):
+        K, V, _ = synth.tiny_chunk(c)
+        out, ws = _gpu_quant(lib, K, V, ws)
+        _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"tiny chunk {c}")
+
+
+@pytest.mark.parametrize("index", [0, 1])
+def test_quantize_only_full_size_bit_exact(lib, orc, index):
+    K, V = synth.quant_chunk(index)
+    out, _ = _gpu_quant(lib, K, V)
+    _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"quantize-only chunk {index}")
+
+
+@pytest.mark.parametrize("T,H", [(1, 2), (48, 2), (63, 3), (65, 1), (136, 4), (200, 5), (1000, 6)])
+def test_ragged_shapes_bit_exact(lib, orc, T, H):
+    K = synth.k_with_offsets_bf16(31, T, H, (T, H, 128), outlier_mult=50.0)
+    V = synth.gaussian_bf16(31, T, H, synth.T_V, (T, H, 128))
+    out, _ = _gpu_quant(lib, K, V)
+    _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"T={T} H={H}")
+
+
+def test_degenerate_inputs_bit_exact(lib, orc):
+    T, H = 100, 2
+    zeros = np.zeros((T, H, 128), np.uint16)
+    rng = np.random.default_rng(3)
+    const = np.repeat(synth.to_bf16_bits(rng.standard_normal((1, H, 128)) * 3), T, axis=0)
+    for K, V, what in ((zeros, zeros, "zeros"), (const, const, "constant channels"),
+                       (const, zeros, "constant K, zero V")):
+        out, _ = _gpu_quant(lib, K, V)
+        _assert_same(out.to_host(), orc.quantize_chunk(K, V), what)
+
+
+def test_repeated_calls_share_one_workspace(lib, orc):
+    ws = None
+    for i in range(3):
+        K = synth.k_with_offsets_bf16(40 + i, 0, 0, (300, 4, 128))
+        V = synth.gaussian_bf16(40 + i, 0, 0, synth.T_V, (300, 4, 128))
+        out, ws = _gpu_quant(lib, K, V, ws)
+        _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"call {i}")
+
+
+@pytest.mark.parametrize("bf16_out", [False, True])
+def test_dequantize_bit_exact(lib, orc, bf16_out):
+    import torch
+    K, V, _ = synth.tiny_chunk(1)
+    T, H, d = K.shape
+    out, _ = _gpu_quant(lib, K, V)
+    dt = torch.bfloat16 if bf16_out else torch.float32
+    Kd = torch.empty((T, H, d), dtype=dt, device="cuda")
+    Vd = torch.empty((T, H, d), dtype=dt, device="cuda")
+    lib.dequantize(out, Kd, Vd)
+    torch.cuda.synchronize()
+    q = orc.quantize_chunk(K, V)
+    Kr, Vr = orc.dequantize_chunk(q)
+    if bf16_out:
+        Kr, Vr = orc.f32_to_bf16(Kr), orc.f32_to_bf16(Vr)
+        Kg = Kd.view(torch.int16).cpu().numpy().view(np.uint16)
+        Vg = Vd.view(torch.int16).cpu().numpy().view(np.uint16)
+    else:
+        Kr, Vr = Kr.view(np.uint32), Vr.view(np.uint32)
+        Kg = Kd.cpu().numpy().view(np.uint32)
+        Vg = Vd.cpu().numpy().view(np.uint32)
+    assert np.array_equal(Kg, Kr) and np.array_equal(Vg, Vr)
+
+
+def test_dequantize_full_size_bit_exact(lib, orc):
+    import torch
+    K, V = synth.quant_chunk(2)
+    T, H, d = K.shape
+    out, _ = _gpu_quant(lib, K, V)
+    Kd = torch.empty((T, H, d), dtype=torch.float32, device="cuda")
+    lib.dequantize(out, K_out=Kd)
+    torch.cuda.synchronize()
+    q = orc.quantize_chunk(K, V)
+    Kr = orc.dequantize_tensor(q["k_codes"], q["k_scales"], q["k_mean"], q["s_k"], T, H, d)
+    assert np.array_equal(Kd.cpu().numpy().view(np.uint32), Kr.view(np.uint32))
