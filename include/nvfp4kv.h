@@ -68,6 +68,12 @@ typedef enum {
     NVFP4KV_ERR_DEVICE_TIMEOUT = 7   /* a kernel's bounded wait gave up */
 } nvfp4kv_status;
 
+/* Element type of an output tensor. */
+typedef enum {
+    NVFP4KV_F32 = 0,     /* IEEE float32 */
+    NVFP4KV_BF16 = 1     /* bfloat16, rounded to nearest even from float32 */
+} nvfp4kv_dtype;
+
 /* Device pointers to one quantized chunk (layouts above). */
 typedef struct {
     uint8_t* k_codes;
@@ -132,7 +138,7 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
 /*
  * De-quantize a chunk back to [T_c][H][d] (device): x = decode(q) *
  * (decode(scale) * s), plus mean for K, each step one fp32 operation.
- * out_dtype 0 = float32 output, 1 = bf16 (the fp32 value rounded to nearest
+ * out_dtype: NVFP4KV_F32 or NVFP4KV_BF16 (the fp32 value rounded to nearest
  * even).  K_out or V_out may be NULL to skip that tensor.
  */
 nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, int d,
@@ -148,15 +154,18 @@ nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, 
  * Method > 算法层设计; fused de-quantization, Method > 推理基础设施).
  *   chunks: host array of n_chunks (1..NVFP4KV_MAX_KEY_CHUNKS) views, each of
  *           T_c tokens, H heads, d = 128.
- *   Q, O:   [T_q][H][d] bf16, device; O is written, Q is read.
+ *   Q:      [T_q][H][d] bf16, device.
+ *   O:      [T_q][H][d] device, written, element type o_dtype (NVFP4KV_F32 or
+ *           NVFP4KV_BF16).
  *   softmax_scale: <= 0 selects 1/sqrt(d).
  *   ws:     workspace as for the quantizer (status word only).
  * Softmax statistics are fp32; the products run on the tensor cores in bf16
- * with the de-quantized values exact in bf16; the result is rounded to bf16.
+ * with the de-quantized values exact in bf16; the normalized result is
+ * stored in o_dtype.
  */
 nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
                                  int T_c, int H, int d, const void* Q, int T_q,
-                                 void* O, float softmax_scale, void* ws,
+                                 void* O, int o_dtype, float softmax_scale, void* ws,
                                  nvfp4kv_stream_t stream);
 
 /* ------------------------------------------------------------------ cache */
@@ -233,12 +242,13 @@ nvfp4kv_status kvcache_advance(kvcache* cache, int layer, nvfp4kv_chunk_view* ou
 
 /*
  * Sink-window attention of `layer`'s queries Q [T_q][H][d] (bf16, device)
- * over its current key set, written to O [T_q][H][d] (bf16, device): the
+ * over its current key set, written to O [T_q][H][d] (device, o_dtype): the
  * key set of kvcache_keyset() passed to nvfp4kv_attention().
  * NVFP4KV_ERR_EMPTY_KEYSET if no chunk is attended.
  */
 nvfp4kv_status sink_window_attention(const kvcache* cache, int layer, const void* Q, int T_q,
-                                     void* O, float softmax_scale, nvfp4kv_stream_t stream);
+                                     void* O, int o_dtype, float softmax_scale,
+                                     nvfp4kv_stream_t stream);
 
 /* The cache's workspace status (see nvfp4kv_workspace_status). */
 nvfp4kv_status kvcache_check_status(kvcache* cache, nvfp4kv_stream_t stream);

@@ -20,6 +20,7 @@ STATUS_NAMES = ["OK", "ERR_INVALID_ARG", "ERR_ALIGNMENT", "ERR_UNSUPPORTED", "ER
                 "ERR_EMPTY_KEYSET", "ERR_CUDA", "ERR_DEVICE_TIMEOUT"]
 MAX_KEY_CHUNKS = 32
 HEAD_DIM = 128
+F32, BF16 = 0, 1              # nvfp4kv_dtype
 
 _lib = None
 
@@ -66,7 +67,7 @@ def load():
         "nvfp4kv_workspace_status": (st, [vp, vp]),
         "nvfp4kv_quantize_chunk": (st, [vp, vp, i32, i32, i32, cv, vp, vp]),
         "nvfp4kv_dequantize": (st, [cv, i32, i32, i32, vp, vp, i32, vp]),
-        "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, f32, vp, vp]),
+        "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp]),
         "kvcache_pool_bytes": (sz, [cfgp]),
         "kvcache_create": (st, [cfgp, vp, vp, ctypes.POINTER(vp)]),
         "kvcache_destroy": (None, [vp]),
@@ -76,7 +77,7 @@ def load():
         "kvcache_num_chunks": (st, [vp, i32, ctypes.POINTER(i64)]),
         "kvcache_chunk_view": (st, [vp, i32, i64, cv]),
         "kvcache_advance": (st, [vp, i32, cv]),
-        "sink_window_attention": (st, [vp, i32, vp, i32, vp, f32, vp]),
+        "sink_window_attention": (st, [vp, i32, vp, i32, vp, i32, f32, vp]),
         "kvcache_check_status": (st, [vp, vp]),
         "nvfp4kv_check_formats": (st, [i32, vp, vp, sz, vp]),
         "nvfp4kv_version": (ctypes.c_char_p, []),
@@ -101,6 +102,15 @@ def _ptr(x):
     if isinstance(x, int):
         return x
     return x.data_ptr()
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"output dtype {t.dtype} is not float32 or bfloat16")
 
 
 def _stream(stream):
@@ -201,9 +211,8 @@ def quantize_chunk(K, V, out: ChunkBuffer, ws, stream=None):
 
 def dequantize(chunk: ChunkBuffer, K_out=None, V_out=None, stream=None):
     """Write de-quantized [T_c, H, d] K and/or V (float32 or bf16 tensors)."""
-    import torch
     t = K_out if K_out is not None else V_out
-    dtype = 1 if t.dtype == torch.bfloat16 else 0
+    dtype = _dtype_code(t)
     _check(load().nvfp4kv_dequantize(ctypes.byref(chunk.view), chunk.T_c, chunk.H, chunk.d,
                                      _ptr(K_out), _ptr(V_out), dtype, _stream(stream)),
            "nvfp4kv_dequantize")
@@ -217,7 +226,8 @@ def attention(chunks, Q, O, ws, softmax_scale=0.0, stream=None):
     T_c = first.T_c if hasattr(first, "T_c") else 0
     T_q, H, d = Q.shape
     _check(load().nvfp4kv_attention(arr, len(views), T_c, H, d, _ptr(Q), T_q, _ptr(O),
-                                    float(softmax_scale), _ptr(ws), _stream(stream)),
+                                    _dtype_code(O), float(softmax_scale), _ptr(ws),
+                                    _stream(stream)),
            "nvfp4kv_attention")
 
 
@@ -296,7 +306,8 @@ class KVCache:
     def attention(self, layer, Q, O, softmax_scale=0.0, stream=None):
         T_q = Q.shape[0]
         _check(load().sink_window_attention(self._h, layer, _ptr(Q), T_q, _ptr(O),
-                                            float(softmax_scale), _stream(stream)),
+                                            _dtype_code(O), float(softmax_scale),
+                                            _stream(stream)),
                "sink_window_attention")
 
     def check_status(self, stream=None) -> int:

@@ -179,7 +179,8 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
 nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, int d,
                                   void* K_out, void* V_out, int out_dtype,
                                   nvfp4kv_stream_t stream) {
-    if (!in || !valid_shape(T_c, H, d) || !view_ok(*in) || (out_dtype != 0 && out_dtype != 1))
+    if (!in || !valid_shape(T_c, H, d) || !view_ok(*in) ||
+        (out_dtype != NVFP4KV_F32 && out_dtype != NVFP4KV_BF16))
         return NVFP4KV_ERR_INVALID_ARG;
     if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
     if ((K_out && !aligned16(K_out)) || (V_out && !aligned16(V_out))) return NVFP4KV_ERR_ALIGNMENT;
@@ -188,10 +189,10 @@ nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, 
 }
 
 nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c, int H,
-                                 int d, const void* Q, int T_q, void* O, float softmax_scale,
-                                 void* ws, nvfp4kv_stream_t stream) {
+                                 int d, const void* Q, int T_q, void* O, int o_dtype,
+                                 float softmax_scale, void* ws, nvfp4kv_stream_t stream) {
     if (!chunks || !Q || !O || !ws || T_q <= 0 || !valid_shape(T_c, H, d) ||
-        !valid_shape(T_q, H, d))
+        !valid_shape(T_q, H, d) || (o_dtype != NVFP4KV_F32 && o_dtype != NVFP4KV_BF16))
         return NVFP4KV_ERR_INVALID_ARG;
     if (n_chunks <= 0) return NVFP4KV_ERR_EMPTY_KEYSET;
     if (n_chunks > NVFP4KV_MAX_KEY_CHUNKS) return NVFP4KV_ERR_CAPACITY;
@@ -201,7 +202,7 @@ nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
     if (!aligned16(Q) || !aligned16(O) || !aligned256(ws)) return NVFP4KV_ERR_ALIGNMENT;
     if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
     if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)d);
-    return launch_attention(chunks, n_chunks, T_c, H, Q, T_q, O, softmax_scale, ws,
+    return launch_attention(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale, ws,
                             (cudaStream_t)stream);
 }
 
@@ -327,7 +328,8 @@ nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const vo
 }
 
 nvfp4kv_status sink_window_attention(const kvcache* cache, int layer, const void* Q, int T_q,
-                                     void* O, float softmax_scale, nvfp4kv_stream_t stream) {
+                                     void* O, int o_dtype, float softmax_scale,
+                                     nvfp4kv_stream_t stream) {
     if (!cache || !Q || !O || T_q <= 0) return NVFP4KV_ERR_INVALID_ARG;
     if (layer < 0 || layer >= cache->cfg.layers) return NVFP4KV_ERR_CAPACITY;
     std::vector<int64_t> ids;
@@ -341,7 +343,7 @@ nvfp4kv_status sink_window_attention(const kvcache* cache, int layer, const void
         views[i] = slot_view(cache, layer, s);
     }
     return nvfp4kv_attention(views, (int)ids.size(), cache->cfg.T_c, cache->cfg.H, cache->cfg.d,
-                             Q, T_q, O, softmax_scale, cache->ws, stream);
+                             Q, T_q, O, o_dtype, softmax_scale, cache->ws, stream);
 }
 
 nvfp4kv_status kvcache_check_status(kvcache* cache, nvfp4kv_stream_t stream) {

@@ -41,7 +41,8 @@ struct AttnArgs {
     ChunkPtrs chunk[NVFP4KV_MAX_KEY_CHUNKS];
     int n_chunks, T_c, H, T_q;
     const uint16_t* Q;
-    uint16_t* O;
+    void* O;
+    int o_f32;                      // 1: float32 output, 0: bf16
     float scale_log2;               // softmax scale * log2(e)
 };
 
@@ -266,12 +267,17 @@ __global__ void __launch_bounds__(kThreads) attention_mma_kernel(const AttnArgs 
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
         const int col = n * 8 + 2 * tq;
-        if (r0 < a.T_q)
-            *reinterpret_cast<uint32_t*>(a.O + ((size_t)r0 * H + h) * kHeadDim + col) =
-                pack_bf16(o[n][0] * i0, o[n][1] * i0);
-        if (r1 < a.T_q)
-            *reinterpret_cast<uint32_t*>(a.O + ((size_t)r1 * H + h) * kHeadDim + col) =
-                pack_bf16(o[n][2] * i1, o[n][3] * i1);
+        const size_t e0 = ((size_t)r0 * H + h) * kHeadDim + col;
+        const size_t e1 = ((size_t)r1 * H + h) * kHeadDim + col;
+        if (a.o_f32) {
+            float* Of = static_cast<float*>(a.O);
+            if (r0 < a.T_q) *reinterpret_cast<float2*>(Of + e0) = make_float2(o[n][0] * i0, o[n][1] * i0);
+            if (r1 < a.T_q) *reinterpret_cast<float2*>(Of + e1) = make_float2(o[n][2] * i1, o[n][3] * i1);
+        } else {
+            uint16_t* Ob = static_cast<uint16_t*>(a.O);
+            if (r0 < a.T_q) *reinterpret_cast<uint32_t*>(Ob + e0) = pack_bf16(o[n][0] * i0, o[n][1] * i0);
+            if (r1 < a.T_q) *reinterpret_cast<uint32_t*>(Ob + e1) = pack_bf16(o[n][2] * i1, o[n][3] * i1);
+        }
     }
 }
 
@@ -281,8 +287,8 @@ constexpr size_t kSmemBytes =
 }  // namespace
 
 nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
-                                    int H, const void* Q, int T_q, void* O, float softmax_scale,
-                                    cudaStream_t stream) {
+                                    int H, const void* Q, int T_q, void* O, int o_dtype,
+                                    float softmax_scale, cudaStream_t stream) {
     static bool configured = false;
     if (!configured) {
         if (cudaFuncSetAttribute(attention_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -304,7 +310,8 @@ nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chun
     a.H = H;
     a.T_q = T_q;
     a.Q = static_cast<const uint16_t*>(Q);
-    a.O = static_cast<uint16_t*>(O);
+    a.O = O;
+    a.o_f32 = o_dtype == NVFP4KV_F32 ? 1 : 0;
     a.scale_log2 = softmax_scale * kLog2e;
     dim3 grid((T_q + kM - 1) / kM, H);
     attention_mma_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a);
@@ -312,10 +319,11 @@ nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chun
 }
 
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c, int H,
-                                const void* Q, int T_q, void* O, float softmax_scale, void* ws,
-                                cudaStream_t stream) {
+                                const void* Q, int T_q, void* O, int o_dtype, float softmax_scale,
+                                void* ws, cudaStream_t stream) {
     (void)ws;
-    return launch_attention_mma(chunks, n_chunks, T_c, H, Q, T_q, O, softmax_scale, stream);
+    return launch_attention_mma(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
+                                stream);
 }
 
 }  // namespace nvfp4kv

@@ -48,11 +48,11 @@ nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,
                                     cudaStream_t stream);
 
 nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
-                                    int H, const void* Q, int T_q, void* O, float softmax_scale,
-                                    cudaStream_t stream);
+                                    int H, const void* Q, int T_q, void* O, int o_dtype,
+                                    float softmax_scale, cudaStream_t stream);
 
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
-                                int H, const void* Q, int T_q, void* O, float softmax_scale,
-                                void* ws, cudaStream_t stream);
+                                int H, const void* Q, int T_q, void* O, int o_dtype,
+                                float softmax_scale, void* ws, cudaStream_t stream);
 
 }  // namespace nvfp4kv

@@ -71,10 +71,11 @@ def test_rejects_bad_arguments_without_device_work(L):
     assert q(FAKE, FAKE, 32, 2, 128, ctypes.byref(cv), FAKE + 16, None) == swv.ERR_ALIGNMENT
     a = L.nvfp4kv_attention
     arr = (swv.ChunkView * 1)(cv)
-    assert a(arr, 0, 32, 2, 128, FAKE, 32, FAKE, 0.0, FAKE, None) == swv.ERR_EMPTY_KEYSET
-    assert a(arr, 33, 32, 2, 128, FAKE, 32, FAKE, 0.0, FAKE, None) == swv.ERR_CAPACITY
-    assert a(arr, 1, 32, 2, 128, FAKE + 4, 32, FAKE, 0.0, FAKE, None) == swv.ERR_ALIGNMENT
-    assert a(arr, 1, 32, 2, 96, FAKE, 32, FAKE, 0.0, FAKE, None) == swv.ERR_UNSUPPORTED
+    assert a(arr, 0, 32, 2, 128, FAKE, 32, FAKE, 1, 0.0, FAKE, None) == swv.ERR_EMPTY_KEYSET
+    assert a(arr, 33, 32, 2, 128, FAKE, 32, FAKE, 1, 0.0, FAKE, None) == swv.ERR_CAPACITY
+    assert a(arr, 1, 32, 2, 128, FAKE + 4, 32, FAKE, 1, 0.0, FAKE, None) == swv.ERR_ALIGNMENT
+    assert a(arr, 1, 32, 2, 96, FAKE, 32, FAKE, 1, 0.0, FAKE, None) == swv.ERR_UNSUPPORTED
+    assert a(arr, 1, 32, 2, 128, FAKE, 32, FAKE, 7, 0.0, FAKE, None) == swv.ERR_INVALID_ARG
     assert L.nvfp4kv_check_formats(9, FAKE, FAKE, 1, None) == swv.ERR_INVALID_ARG
     assert L.nvfp4kv_workspace_init(None, 256, None) == swv.ERR_INVALID_ARG
 
@@ -157,7 +158,7 @@ def test_cache_rejects_bad_layers_and_sizes(L):
     assert L.kvcache_advance(h, -1, ctypes.byref(v)) == swv.ERR_CAPACITY
     assert L.kvcache_rebind_shot_sink(h, -3) == swv.ERR_INVALID_ARG
     # no chunk yet: nothing to attend, reported before any launch
-    assert L.sink_window_attention(h, 0, FAKE, 32, FAKE, 0.0, None) == swv.ERR_EMPTY_KEYSET
+    assert L.sink_window_attention(h, 0, FAKE, 32, FAKE, 1, 0.0, None) == swv.ERR_EMPTY_KEYSET
     L.kvcache_destroy(h)
     cfg = swv.KVCacheConfig(1, 2, 128, 32, 20, 10, 10)
     hh = ctypes.c_void_p()

@@ -13,12 +13,24 @@ pytestmark = pytest.mark.gpu
 
 
 def _attend(lib, cache, layer, Q):
+    """Both output types: (float32 output, bf16 output) as float64 arrays."""
     import torch
-    O = torch.empty((Q.shape[0],) + Q.shape[1:], dtype=torch.bfloat16, device="cuda")
-    cache.attention(layer, dev_bf16(Q), O)
-    torch.cuda.synchronize()
-    assert cache.check_status() == lib.OK
-    return host_bf16_to_f64(O)
+    outs = []
+    for dt in (torch.float32, torch.bfloat16):
+        O = torch.empty((Q.shape[0],) + Q.shape[1:], dtype=dt, device="cuda")
+        cache.attention(layer, dev_bf16(Q), O)
+        torch.cuda.synchronize()
+        assert cache.check_status() == lib.OK
+        outs.append(host_bf16_to_f64(O))
+    return outs
+
+
+def _close_both(outs, ref, what, rows=None):
+    o32, o16 = outs
+    if rows is not None:
+        o32, o16 = o32[rows], o16[rows]
+    assert_attention_close(o32, ref, what + " (fp32 output)")
+    assert_attention_close(o16, ref, what + " (bf16 output)", bf16_output=True)
 
 
 def test_tiny_config_rollout(lib, orc):
@@ -33,7 +45,7 @@ def test_tiny_config_rollout(lib, orc):
         assert ids == orc.keyset(n + 1, c["S_g"], c["S_s"], c["W"], 0)
         out = _attend(lib, cache, 0, Q)
         ref = orc.attention_f64([qs[i] for i in ids], Q)
-        assert_attention_close(out, ref, f"tiny chunk {n}")
+        _close_both(out, ref, f"tiny chunk {n}")
 
 
 def test_one_layer_attention_full_size(lib, orc):
@@ -54,7 +66,7 @@ def test_one_layer_attention_full_size(lib, orc):
     out = _attend(lib, cache, 0, Q)
     rows = sample_rows(c["T_c"], n_random=24, seed=2)
     ref = orc.attention_f64([qs[i] for i in want_ids], Q, rows=rows)
-    assert_attention_close(out[rows], ref, "one-layer attention")
+    _close_both(out, ref, "one-layer attention", rows=rows)
 
 
 @pytest.mark.parametrize("T_c,T_q,H", [(48, 100, 2), (136, 136, 3), (200, 7, 2), (1, 5, 2),
@@ -72,10 +84,13 @@ def test_ragged_shapes(lib, orc, T_c, T_q, H):
         chunks.append(buf)
         qs.append(orc.quantize_chunk(K, V))
     Q = synth.gaussian_bf16(60, T_c, H, synth.T_Q, (T_q, H, 128))
-    O = torch.empty((T_q, H, 128), dtype=torch.bfloat16, device="cuda")
-    lib.attention(chunks, dev_bf16(Q), O, ws)
-    torch.cuda.synchronize()
-    assert_attention_close(host_bf16_to_f64(O), orc.attention_f64(qs, Q), f"T_c={T_c} T_q={T_q}")
+    ref = orc.attention_f64(qs, Q)
+    for dt in (torch.float32, torch.bfloat16):
+        O = torch.empty((T_q, H, 128), dtype=dt, device="cuda")
+        lib.attention(chunks, dev_bf16(Q), O, ws)
+        torch.cuda.synchronize()
+        assert_attention_close(host_bf16_to_f64(O), ref, f"T_c={T_c} T_q={T_q} {dt}",
+                               bf16_output=dt == torch.bfloat16)
 
 
 def test_duplicated_list_counts_twice(lib, orc):
@@ -92,7 +107,7 @@ def test_duplicated_list_counts_twice(lib, orc):
         bufs.append(b)
         qs.append(orc.quantize_chunk(K, V))
     _, _, Q = synth.tiny_chunk(3)
-    O = torch.empty(Q.shape, dtype=torch.bfloat16, device="cuda")
+    O = torch.empty(Q.shape, dtype=torch.float32, device="cuda")
     lib.attention([bufs[0], bufs[0], bufs[1]], dev_bf16(Q), O, ws)
     torch.cuda.synchronize()
     out = host_bf16_to_f64(O)
@@ -115,7 +130,7 @@ def test_window_zero_is_sink_only(lib, orc):
         qs[n] = orc.quantize_chunk(K, V)
     assert cache.keyset(0) == [0, 2]
     out = _attend(lib, cache, 0, Q)
-    assert_attention_close(out, orc.attention_f64([qs[0], qs[2]], Q), "W=0")
+    _close_both(out, orc.attention_f64([qs[0], qs[2]], Q), "W=0")
 
 
 def test_overlapping_sinks_deduplicated(lib, orc):
@@ -129,7 +144,7 @@ def test_overlapping_sinks_deduplicated(lib, orc):
     # A_g = {0,1}, A_s = {0,1} (shot 0), window = {2,3}
     assert cache.keyset(0) == [0, 1, 2, 3]
     out = _attend(lib, cache, 0, Q)
-    assert_attention_close(out, orc.attention_f64([qs[i] for i in range(4)], Q), "dedup")
+    _close_both(out, orc.attention_f64([qs[i] for i in range(4)], Q), "dedup")
 
 
 def test_empty_keyset_is_an_error(lib):
