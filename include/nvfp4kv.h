@@ -136,6 +136,34 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
                                       nvfp4kv_stream_t stream);
 
 /*
+ * nvfp4kv_quantize_chunk without a workspace argument, for callers that are
+ * not allowed to allocate device memory: an inference engine that owns every
+ * byte of the GPU and gives its plugins no scratch space, or a real-time loop
+ * that must not call cudaMalloc because an allocation can synchronize the
+ * device and stall the other streams.  The paper has no counterpart to this
+ * entry point; it is a deployment convenience.
+ *
+ * The scratch (partial sums, maxima, barrier and status words) lives in one
+ * 4 MiB array compiled into the library, which every GPU that loads the
+ * library holds until the process exits.  Chunks whose scratch,
+ * 256 + ceil(T_c/64)*H*d*8 (rounded up to 256) + 32768 bytes, exceeds 4 MiB
+ * are refused with NVFP4KV_ERR_CAPACITY before any device work (H = 24,
+ * d = 128 allows T_c up to 10,816).  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  Every call
+ * clears the barrier and status words on `stream` and then reuses the same
+ * array, so calls that overlap on the GPU (other streams, other threads)
+ * race; the array keeps the last call's contents.  A kernel-side timeout is
+ * not reported here; use nvfp4kv_quantize_chunk with a workspace to read it.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * Output, arguments and other errors are those of nvfp4kv_quantize_chunk,
+ * bit for bit.
+ */
+nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const void* V, int T_c, int H,
+                                              int d, const nvfp4kv_chunk_view* out,
+                                              nvfp4kv_stream_t stream);
+
+/*
  * De-quantize a chunk back to [T_c][H][d] (device): x = decode(q) *
  * (decode(scale) * s), plus mean for K, each step one fp32 operation.
  * out_dtype: NVFP4KV_F32 or NVFP4KV_BF16 (the fp32 value rounded to nearest

@@ -468,3 +468,68 @@ nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,
 }
 
 }  // namespace nvfp4kv
+
+// ---------------------------------------------------------------- no-allocation entry point
+//
+// The same quantization for callers that cannot allocate device memory: the
+// scratch lives in one array compiled into the library.  Host code only sees
+// a stand-in for that array's name; its device address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+#include <mutex>
+
+namespace nvfp4kv {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;    // 4 MiB per GPU
+
+static __device__ __align__(256) unsigned char g_quant_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[64];       // device address of g_quant_scratch, per device ordinal
+}  // namespace
+
+}  // namespace nvfp4kv
+
+extern "C" nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const void* V, int T_c,
+                                                         int H, int d,
+                                                         const nvfp4kv_chunk_view* out,
+                                                         nvfp4kv_stream_t stream) {
+    using namespace nvfp4kv;
+    if (!K || !V || !out || T_c <= 0 || H <= 0 || T_c > (1 << 24) || H > 4096 ||
+        !out->k_codes || !out->k_scales || !out->v_codes || !out->v_scales || !out->k_mean ||
+        !out->tensor_scales)
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDim) return NVFP4KV_ERR_UNSUPPORTED;
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) |
+                          reinterpret_cast<uintptr_t>(out->k_codes) |
+                          reinterpret_cast<uintptr_t>(out->v_codes) |
+                          reinterpret_cast<uintptr_t>(out->k_scales) |
+                          reinterpret_cast<uintptr_t>(out->v_scales) |
+                          reinterpret_cast<uintptr_t>(out->k_mean);
+    if ((mis & 15u) != 0 || (reinterpret_cast<uintptr_t>(out->tensor_scales) & 7u) != 0)
+        return NVFP4KV_ERR_ALIGNMENT;
+    // the chunk's scratch must fit the compiled-in array
+    if (ws_layout(T_c, H).total > kStaticScratchBytes) return NVFP4KV_ERR_CAPACITY;
+
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4KV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return NVFP4KV_ERR_CUDA;
+    if (major != 10) return NVFP4KV_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mutex);
+        if (g_scratch_addr[dev] == nullptr) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_quant_scratch) != cudaSuccess || p == nullptr)
+                return NVFP4KV_ERR_CUDA;
+            g_scratch_addr[dev] = p;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    // the grid barrier and the status word must start at zero; the partial
+    // sums and maxima are written before they are read
+    if (cudaMemsetAsync(scratch, 0, sizeof(Control), (cudaStream_t)stream) != cudaSuccess)
+        return NVFP4KV_ERR_CUDA;
+    return launch_quantize(K, V, T_c, H, *out, scratch, (cudaStream_t)stream);
+}

@@ -1,0 +1,65 @@
+"""nvfp4kv_quantize_chunk_noalloc -- the quantizer for callers that may not
+allocate device memory (engines that own all GPU memory and give plugins no
+scratch, real-time loops that must not risk cudaMalloc's synchronization).  It
+keeps its scratch in an array compiled into the library instead of a caller
+workspace.  Checked through the C ABI against nvfp4kv_quantize_chunk (the
+workspace entry point), bit for bit, on two calls in a row; this file is
+collected last so that a failure here comes after every other test ran."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import synth
+from gpu_util import dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _entry(lib):
+    L = lib.load()
+    fn = L.nvfp4kv_quantize_chunk_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                   ctypes.POINTER(lib.ChunkView), ctypes.c_void_p]
+    return fn
+
+
+def _parts(buf):
+    return {k: getattr(buf, k).cpu().numpy()
+            for k in ("k_codes", "k_scales", "v_codes", "v_scales", "k_mean", "tensor_scales")}
+
+
+def test_noalloc_matches_workspace_entry_point_twice(lib):
+    import torch
+    fn = _entry(lib)
+    stream = torch.cuda.current_stream().cuda_stream
+    inputs = [synth.quant_chunk(0), synth.layer_chunk(synth.MULTISHOT, 0, 3)[:2]]
+    for call, (K, V) in enumerate(inputs):
+        T, H, d = K.shape
+        Kd, Vd = dev_bf16(K), dev_bf16(V)
+        ref = lib.ChunkBuffer(T, H, d)
+        ws = lib.new_workspace(T, H, d)
+        lib.quantize_chunk(Kd, Vd, ref, ws)
+        got = lib.ChunkBuffer(T, H, d)
+        st = fn(Kd.data_ptr(), Vd.data_ptr(), T, H, d, ctypes.byref(got.view), stream)
+        assert st == lib.OK, f"call {call}: status {st}"
+        torch.cuda.synchronize()
+        assert lib.workspace_status(ws) == lib.OK
+        a, b = _parts(got), _parts(ref)
+        for k in a:
+            assert np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)), f"call {call}: {k}"
+
+
+def test_noalloc_refuses_chunks_beyond_its_scratch(lib):
+    import torch
+    fn = _entry(lib)
+    K = torch.zeros((16, 2, 128), dtype=torch.bfloat16, device="cuda")
+    buf = lib.ChunkBuffer(16, 2)
+    # 10,880 tokens x 24 heads needs more than the 4 MiB compiled-in scratch;
+    # refused from the sizes alone, before anything reads K
+    st = fn(K.data_ptr(), K.data_ptr(), 10880, 24, 128, ctypes.byref(buf.view),
+            torch.cuda.current_stream().cuda_stream)
+    assert st == lib.ERR_CAPACITY
+    assert fn(K.data_ptr(), K.data_ptr(), 16, 2, 64, ctypes.byref(buf.view), None) \
+        == lib.ERR_UNSUPPORTED
