@@ -15,6 +15,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -121,6 +122,22 @@ bool have_sm100() {
 }
 
 }  // namespace
+
+namespace nvfp4kv {
+nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c, int H,
+                                const void* Q, int T_q, void* O, int o_dtype, float softmax_scale,
+                                void* ws, cudaStream_t stream) {
+    static const bool use_mma = [] {
+        const char* e = std::getenv("NVFP4KV_ATTENTION_KERNEL");
+        return e != nullptr && std::strcmp(e, "mma") == 0;
+    }();
+    if (use_mma)
+        return launch_attention_mma(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
+                                    stream);
+    return launch_attention_tc(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale, ws,
+                               stream);
+}
+}  // namespace nvfp4kv
 
 extern "C" {
 

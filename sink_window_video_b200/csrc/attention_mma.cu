@@ -318,12 +318,6 @@ nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chun
     return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
-nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c, int H,
-                                const void* Q, int T_q, void* O, int o_dtype, float softmax_scale,
-                                void* ws, cudaStream_t stream) {
-    (void)ws;
-    return launch_attention_mma(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
-                                stream);
-}
+
 
 }  // namespace nvfp4kv

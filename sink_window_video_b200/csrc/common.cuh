@@ -20,17 +20,35 @@ constexpr float kTensorScaleDiv = 2688.0f;   // 6 * 448
 // Status bits recorded by kernels in the workspace.
 constexpr unsigned kStatusTimeout = 1u;
 
-// Upper bound on polls of any spin-wait before the kernel gives up, records
-// kStatusTimeout and returns (each poll sleeps ~100 ns: well under a second).
-constexpr long long kSpinLimit = 1ll << 23;
+// Time limit of any single wait inside a kernel, in nanoseconds; a wait that
+// reaches it records kStatusTimeout (and its site) and the kernel returns.
+constexpr unsigned long long kWaitLimitNs = 200ull * 1000 * 1000;
 
 // First 256 bytes of every workspace.
 struct Control {
     unsigned status;      // OR of kStatus* bits; cleared by the host
     unsigned bar_count;   // grid barrier: CTAs arrived at the current barrier
     unsigned bar_gen;     // grid barrier: generation, bumped by the last arrival
-    unsigned pad[61];
+    unsigned diag[4];     // first wait that gave up: site, block (x | y << 16), step, phase
+    unsigned pad[57];
 };
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Record a wait that gave up: the status bit, and the first such site.
+__device__ __forceinline__ void record_timeout(Control* ctl, unsigned site, unsigned step,
+                                               unsigned phase) {
+    atomicOr(&ctl->status, kStatusTimeout);
+    if (atomicCAS(&ctl->diag[0], 0u, site) == 0u) {
+        ctl->diag[1] = blockIdx.x | (blockIdx.y << 16);
+        ctl->diag[2] = step;
+        ctl->diag[3] = phase;
+    }
+}
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
@@ -60,10 +78,10 @@ __device__ __forceinline__ bool grid_barrier(Control* ctl) {
             __threadfence();
             st_release_gpu(&ctl->bar_gen, gen + 1);
         } else {
-            long long spins = 0;
+            const unsigned long long t0 = globaltimer_ns();
             while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
-                if (++spins > kSpinLimit) {
-                    atomicOr(&ctl->status, kStatusTimeout);
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    record_timeout(ctl, 100u, gen, 0u);
                     ok = 0;
                     break;
                 }

@@ -51,6 +51,12 @@ nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chun
                                     int H, const void* Q, int T_q, void* O, int o_dtype,
                                     float softmax_scale, cudaStream_t stream);
 
+nvfp4kv_status launch_attention_tc(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                   int H, const void* Q, int T_q, void* O, int o_dtype,
+                                   float softmax_scale, void* ws, cudaStream_t stream);
+
+// Sink-window attention: the tcgen05 kernel, or the mma.sync kernel when the
+// environment variable NVFP4KV_ATTENTION_KERNEL=mma selects it (cross-checks).
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                 int H, const void* Q, int T_q, void* O, int o_dtype,
                                 float softmax_scale, void* ws, cudaStream_t stream);
