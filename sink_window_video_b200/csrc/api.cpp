@@ -127,14 +127,19 @@ namespace nvfp4kv {
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c, int H,
                                 const void* Q, int T_q, void* O, int o_dtype, float softmax_scale,
                                 void* ws, cudaStream_t stream) {
-    static const bool use_mma = [] {
+    static const int which = [] {
         const char* e = std::getenv("NVFP4KV_ATTENTION_KERNEL");
-        return e != nullptr && std::strcmp(e, "mma") == 0;
+        if (e != nullptr && std::strcmp(e, "mma") == 0) return 1;
+        if (e != nullptr && std::strcmp(e, "tc1") == 0) return 2;
+        return 0;
     }();
-    if (use_mma)
+    if (which == 1)
         return launch_attention_mma(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
                                     stream);
-    return launch_attention_tc(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale, ws,
+    if (which == 2)
+        return launch_attention_tc(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
+                                   ws, stream);
+    return launch_attention_ws(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale, ws,
                                stream);
 }
 }  // namespace nvfp4kv

@@ -1,0 +1,576 @@
+// attention_ws.cu -- warp-specialized sink-window attention over the NVFP4
+// cache on the sm_100a tensor cores (tcgen05), two query tiles in ping-pong.
+//
+// Method ("2605-LongLive2" DeepRead page, Method > 算法层设计: attention over
+// K_eff = A_g u A_s u KV[t-W, t); Method > 推理基础设施: the NVFP4 cache is
+// de-quantized inside the attention kernel):
+//   O = softmax(scale Q K_hat^T) V_hat,  K_hat = q*sb*s_K + mean,  V_hat = q*sb*s_V,
+// computed as in attention_tc.cu: the de-quantized codes q*sb are exact fp16
+// tensor-core operands, s_K and the K-smoothing bias Q.mean_c enter the fp32
+// logits, s_V/s_Vmax scales P per chunk, and Q rows are scaled by powers of two
+// into fp16 range.
+//
+// One CTA per SM: a head and 256 query rows (two 128-row tiles Q0, Q1), keys
+// in 64-key tiles.  Warp roles (352 threads; 11 warps keep 168 registers per
+// thread, registers being split among the four SM sub-partitions):
+//   warps 0-3   softmax of Q0 (thread = row = TMEM lane)
+//   warps 4-7   softmax of Q1
+//   warp 8      tensor memory allocation and the MMA issue (one thread)
+//   warps 9-10  de-quantize K and V tiles (thread = key row) into a 4-stage
+//               shared-memory ring (128-byte-swizzled: K-major B of
+//               S = Q K^T, MN-major B of P V)
+// (warp w runs on SM sub-partition w mod 4: each carries two softmax warps,
+// and the issue and conversion work of the other roles is spread over three.)
+// Tensor memory (512 columns): Q0 | Q1 (fp16, 64 each; the A operand of
+// S = Q K^T) | S0 | S1 (fp32, 64 each; P in fp16 over their first 32) |
+// O0 | O1 (fp32, 128 each).  With Q in tensor memory the MMAs read only B
+// from shared memory, which leaves shared-memory bandwidth for the
+// de-quantization stores.
+// MMA order per key tile t:  PV0(t) QK0(t+1) | PV1(t) QK1(t+1); while one
+// softmax group works on S_i, the tensor core runs the other group's
+// products.  P_i over S_i is safe because tcgen05 MMAs of one thread execute
+// in issue order.
+// Synchronization is by mbarriers only: kv_full/kv_empty (ring), s_full
+// (S_i ready; its commit also covers the previous PV_i, so O_i is quiescent
+// for a rescale), p_full (P_i written), q_ready, o_final.  Every wait is
+// bounded in time and gives up at once when another warp has given up; all
+// decisions ahead of warp-collective tensor-memory instructions are
+// warp-uniform.  On a timeout the kernel records its site in the workspace,
+// drains its MMAs (bounded), frees tensor memory and returns.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace nvfp4kv {
+using namespace tc;
+namespace {
+
+constexpr int kKeysW = 64;                  // keys per tile
+constexpr int kStages = 4;                  // de-quantized K/V ring depth
+constexpr int kThreadsW = 352;
+constexpr int kMmaWarp = 8;
+constexpr int kDequantWarp0 = 9;
+constexpr uint32_t kColQ = 0, kColS = 128, kColO = 256, kColsW = 512;
+constexpr int kStageBytes = kKeysW * 128 * 2;            // 16 KB per operand tile
+constexpr size_t kSmemW = 2 * kStages * kStageBytes + 1024;
+constexpr float kLog2eW = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct WsChunk {
+    const uint8_t* k_codes;
+    const uint8_t* k_scales;
+    const uint8_t* v_codes;
+    const uint8_t* v_scales;
+    const float* k_mean;
+    const float* tensor_scales;
+};
+
+struct WsArgs {
+    WsChunk chunk[NVFP4KV_MAX_KEY_CHUNKS];
+    int n_chunks, T_c, H, T_q;
+    const uint16_t* Q;
+    void* O;
+    int o_f32;
+    float scale_log2;
+    Control* ctl;
+};
+
+struct WsShared {
+    uint64_t kv_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t q_ready[2];
+    uint64_t o_final;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Bounded wait that also gives up as soon as any warp of the CTA gave up.
+// It polls try_wait (which itself suspends the thread for a short while)
+// without sleeping in between: a sleep here delays the wake-up of the
+// critical-path waits by hundreds of cycles.
+__device__ __forceinline__ bool wait_or_abort(uint32_t mbar, uint32_t parity, volatile int* abort,
+                                              Control* ctl, unsigned site, unsigned step) {
+    if (mbar_try_wait(mbar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait(mbar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            record_timeout(ctl, site, step, parity);
+            return false;
+        }
+    }
+}
+
+// K-major, 64-key, 128-byte-swizzled operand: key row kl, 16-byte chunk c of
+// d (0..15).  Two 8 KB blocks along d.
+__device__ __forceinline__ uint32_t kv_off(int kl, int c) {
+    return (uint32_t)((c >> 3) * 8192 + kl * 128 + (((c & 7) ^ (kl & 7)) << 4));
+}
+
+// De-quantize 64 consecutive codes (32 bytes) with their 4 block scales into
+// chunks 8*half .. 8*half+7 of key row kl of a swizzled tile.
+__device__ __forceinline__ void dequant_half(const uint4 c0, const uint4 c1, uint32_t sc,
+                                             uint8_t* tile, int kl, int half) {
+    const uint32_t s01 = cvt_e4m3x2_to_f16x2(sc & 0xFFFFu);
+    const uint32_t s23 = cvt_e4m3x2_to_f16x2(sc >> 16);
+    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {            // block b: code words 2b, 2b+1
+        const uint32_t pair = (b < 2) ? s01 : s23;
+        const uint32_t sh = (b & 1) ? (pair >> 16) : (pair & 0xFFFFu);
+        const uint32_t s2 = sh | (sh << 16);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint32_t h[4];
+            cvt_e2m1x8_to_f16x2(cw[2 * b + w], h);
+            uint4 o;
+            o.x = hmul2_u32(h[0], s2);
+            o.y = hmul2_u32(h[1], s2);
+            o.z = hmul2_u32(h[2], s2);
+            o.w = hmul2_u32(h[3], s2);
+            *reinterpret_cast<uint4*>(tile + kv_off(kl, half * 8 + 2 * b + w)) = o;
+        }
+    }
+}
+
+// 2^x for a pair on the FMA and integer pipes (the special-function unit is
+// shared by two softmax warps per sub-partition and is the scarcer resource):
+// n = round(x) by adding and subtracting 1.5*2^23, f = x - n in [-1/2, 1/2],
+// 2^f by a cubic (least-squares fit on relative error, max 7.5e-5), and 2^n
+// added to the exponent field.  x is clamped to -126 so 2^n stays normal;
+// inputs here are at most 8 (the lazy-max bound).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+    float2 p = __ffma2_rn(make_float2(0.055170949548482895f, 0.055170949548482895f), f,
+                          make_float2(0.2426096349954605f, 0.2426096349954605f));
+    p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = __ffma2_rn(p, f, make_float2(0.9999281764030457f, 0.9999281764030457f));
+    float2 r;
+    r.x = __int_as_float(__float_as_int(p.x) + ((__float_as_int(t.x) - 0x4B400000) << 23));
+    r.y = __int_as_float(__float_as_int(p.y) + ((__float_as_int(t.y) - 0x4B400000) << 23));
+    return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ WsShared sh;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int h = blockIdx.y;
+    const int m0 = blockIdx.x * 256;
+    const int H = a.H, T_c = a.T_c;
+    const int tiles_per_chunk = (T_c + kKeysW - 1) / kKeysW;
+    const int ntiles = a.n_chunks * tiles_per_chunk;
+    volatile int* abort = &sh.abort;
+
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* Kt = base;                                  // [kStages][16 KB]
+    uint8_t* Vt = base + kStages * kStageBytes;          // [kStages][16 KB]
+
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sh.tmem_base)),
+                     "r"(kColsW));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        sh.abort = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&sh.kv_full[s]), 64);
+            mbar_init(smem_u32(&sh.kv_empty[s]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&sh.s_full[i]), 1);
+            mbar_init(smem_u32(&sh.p_full[i]), 128);
+            mbar_init(smem_u32(&sh.q_ready[i]), 128);
+        }
+        mbar_init(smem_u32(&sh.o_final), 1);
+        mbar_init(smem_u32(&sh.drain), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ softmax
+        const int qi = warp >> 2;                          // query tile 0 or 1
+        const int r = tid & 127;                           // row in the tile
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tQ = tmem + lane_base + kColQ + 64u * qi;
+        const uint32_t tS = tmem + lane_base + kColS + 64u * qi;
+        const uint32_t tO = tmem + lane_base + kColO + 128u * qi;
+        const int row = m0 + qi * 128 + r;
+        const bool rvalid = row < a.T_q;
+        const uint4* qsrc = reinterpret_cast<const uint4*>(a.Q + ((size_t)row * H + h) * kHeadDim);
+
+        // Q row -> fp16 (scaled by 2^-e into range) -> tensor memory (A of Q K^T)
+        float qexp;
+        {
+            uint4 w[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) w[c] = rvalid ? qsrc[c] : make_uint4(0, 0, 0, 0);
+            uint32_t amax_bits = 0;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    amax_bits = max(amax_bits, (u[j] << 16) & 0x7FFFFFFFu);
+                    amax_bits = max(amax_bits, u[j] & 0x7FFF0000u);
+                }
+            }
+            int e = 0;
+            if (amax_bits != 0) e = max(-120, min(120, (int)(amax_bits >> 23) - 127 - 14));
+            const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+            qexp = __uint_as_float((uint32_t)(127 + e) << 23);
+            uint32_t qh[64];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                float f[8];
+                unpack_bf16x8(w[c], f);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) qh[4 * c + j] = pack_f16x2(f[2 * j] * down, f[2 * j + 1] * down);
+            }
+            tmem_st32(tQ, qh);
+            tmem_st32(tQ + 32, qh + 32);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sh.q_ready[qi]));
+
+        float sVmax = 0.0f;
+        for (int ci = 0; ci < a.n_chunks; ++ci) sVmax = fmaxf(sVmax, a.chunk[ci].tensor_scales[1]);
+
+        float m_run = -INFINITY, l_run = 0.0f;
+        bool o_written = false, ok = true;
+        int t = 0;
+        const uint32_t s_full = smem_u32(&sh.s_full[qi]);
+        const uint32_t p_full = smem_u32(&sh.p_full[qi]);
+        for (int ci = 0; ci < a.n_chunks && ok; ++ci) {
+            const WsChunk cp = a.chunk[ci];
+            const float sK = cp.tensor_scales[0], sV = cp.tensor_scales[1];
+            float qmu = 0.0f;
+            if (rvalid) {
+                const float4* mp = reinterpret_cast<const float4*>(cp.k_mean + h * kHeadDim);
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c) {
+                    float f[8];
+                    unpack_bf16x8(qsrc[c], f);
+                    const float4 u0 = mp[2 * c], u1 = mp[2 * c + 1];
+                    qmu = fmaf(f[0], u0.x, qmu); qmu = fmaf(f[1], u0.y, qmu);
+                    qmu = fmaf(f[2], u0.z, qmu); qmu = fmaf(f[3], u0.w, qmu);
+                    qmu = fmaf(f[4], u1.x, qmu); qmu = fmaf(f[5], u1.y, qmu);
+                    qmu = fmaf(f[6], u1.z, qmu); qmu = fmaf(f[7], u1.w, qmu);
+                }
+            }
+            const float alpha = qexp * sK * a.scale_log2;
+            const float beta = qmu * a.scale_log2;
+            const float lrV = __log2f(sV / sVmax);
+            const float inv_rV = sVmax / sV;
+            const float2 alpha2 = make_float2(alpha, alpha);
+
+            for (int j0 = 0; j0 < T_c; j0 += kKeysW, ++t) {
+                bool got = wait_or_abort(s_full, (uint32_t)(t & 1), abort, a.ctl, 10u + qi, t);
+                if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t s[64];
+                __syncwarp();
+                tmem_ld32(tS, s);
+                tmem_ld32(tS + 32, s + 32);
+                tmem_wait_ld();
+                const int valid = min(kKeysW, T_c - j0);
+                if (valid < kKeysW) {
+#pragma unroll
+                    for (int k = 0; k < 64; ++k)
+                        if (k >= valid) s[k] = __float_as_uint(-INFINITY);
+                }
+                // row max: eight independent chains, then a short tree
+                float m8[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) m8[c] = fmaxf(__uint_as_float(s[c]), __uint_as_float(s[c + 8]));
+#pragma unroll
+                for (int k = 16; k < 64; k += 16)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        m8[c] = fmax3(m8[c], __uint_as_float(s[k + c]), __uint_as_float(s[k + 8 + c]));
+                float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                                 fmaxf(m8[6], m8[7]));
+                mx = fmaf(mx, alpha, beta);                 // alpha > 0: same argmax
+                const bool grow = mx > m_run + kRescaleLog2 || m_run == -INFINITY;
+                float corr = 1.0f;
+                if (grow) {
+                    const float m_new = fmaxf(mx, m_run);
+                    corr = ex2f(m_run - m_new);
+                    l_run *= corr;
+                    m_run = m_new;
+                }
+                if (o_written && __any_sync(0xFFFFFFFFu, grow)) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + 32 * q, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+                        tmem_st32(tO + 32 * q, ov);
+                    }
+                }
+                // p' = 2^(logit - m + log2(s_V/s_Vmax)), one fused multiply-add each
+                // two of every eight pairs on the FMA pipe, the rest on the
+                // special-function unit; four independent partial sums
+                const float b2 = beta - m_run + lrV;
+                const float2 b22 = make_float2(b2, b2);
+                float2 acc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                                 make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+                uint32_t p[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    float2 z = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])),
+                                          alpha2, b22);
+                    if ((k & 7) >= 6) {
+                        z = ex2_poly2(z);
+                    } else {
+                        z.x = ex2f(z.x);
+                        z.y = ex2f(z.y);
+                    }
+                    acc[k & 3] = __fadd2_rn(acc[k & 3], z);
+                    p[k] = pack_f16x2(z.x, z.y);
+                }
+                __syncwarp();
+                tmem_st32(tS, p);
+                tmem_wait_st();
+                const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+                const float2 a03 = __fadd2_rn(a01, a23);
+                l_run += (a03.x + a03.y) * inv_rV;
+                tc_fence_before();
+                mbar_arrive(p_full);
+                o_written = true;
+            }
+        }
+        if (ok) {
+            bool got = wait_or_abort(smem_u32(&sh.o_final), 0u, abort, a.ctl, 20u + qi, ntiles);
+            ok = __all_sync(0xFFFFFFFFu, got);
+        }
+        if (ok) {
+            tc_fence_after();
+            const float inv = sVmax / l_run;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t ov[32];
+                __syncwarp();                  // converged for the collective load
+                tmem_ld32(tO + 32 * q, ov);
+                tmem_wait_ld();
+                if (rvalid) {
+                    const size_t o = ((size_t)row * H + h) * kHeadDim + 32 * q;
+                    if (a.o_f32) {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.O) + o);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            dst[c] = make_float4(__uint_as_float(ov[4 * c]) * inv, __uint_as_float(ov[4 * c + 1]) * inv,
+                                                 __uint_as_float(ov[4 * c + 2]) * inv, __uint_as_float(ov[4 * c + 3]) * inv);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.O) + o);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                __nv_bfloat162 b2v = __floats2bfloat162_rn(__uint_as_float(ov[8 * c + 2 * j]) * inv,
+                                                                           __uint_as_float(ov[8 * c + 2 * j + 1]) * inv);
+                                w4[j] = *reinterpret_cast<uint32_t*>(&b2v);
+                            }
+                            dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
+                }
+            }
+        }
+    } else if (warp >= kDequantWarp0) {
+        // ------------------------------------------------------------ de-quantize
+        // One thread per key row; the codes and scales of tile t+1 are loaded
+        // into registers before tile t is converted, so the L2 latency of the
+        // loads overlaps one tile period.
+        const int kl = tid - kDequantWarp0 * 32;           // key row 0..63
+        struct Packed {
+            uint4 kc[4], vc[4];
+            uint2 ks, vs;
+        };
+        auto load_tile = [&](int t, Packed& p) {
+            const int ci = t / tiles_per_chunk;
+            const int key = (t - ci * tiles_per_chunk) * kKeysW + kl;
+            if (t < ntiles && key < T_c) {
+                const WsChunk& cp = a.chunk[ci];
+                const size_t rowi = (size_t)h * T_c + key;
+                const uint4* kp = reinterpret_cast<const uint4*>(cp.k_codes + rowi * 64);
+                const uint4* vp = reinterpret_cast<const uint4*>(cp.v_codes + rowi * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { p.kc[i] = kp[i]; p.vc[i] = vp[i]; }
+                p.ks = *reinterpret_cast<const uint2*>(cp.k_scales + rowi * 8);
+                p.vs = *reinterpret_cast<const uint2*>(cp.v_scales + rowi * 8);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) p.kc[i] = p.vc[i] = make_uint4(0, 0, 0, 0);
+                p.ks = p.vs = make_uint2(0, 0);
+            }
+        };
+        Packed cur, nxt;
+        load_tile(0, cur);
+        for (int t = 0; t < ntiles; ++t) {
+            const int st = t % kStages;
+            load_tile(t + 1, nxt);
+            if (t >= kStages) {
+                bool got = wait_or_abort(smem_u32(&sh.kv_empty[st]),
+                                         (uint32_t)(((t / kStages) - 1) & 1), abort, a.ctl, 30u, t);
+                if (!__all_sync(0xFFFFFFFFu, got)) break;
+            }
+            uint8_t* kt = Kt + st * kStageBytes;
+            uint8_t* vt = Vt + st * kStageBytes;
+            // rows past the chunk's end are zero codes and zero scales: exact zeros
+            dequant_half(cur.kc[0], cur.kc[1], cur.ks.x, kt, kl, 0);
+            dequant_half(cur.kc[2], cur.kc[3], cur.ks.y, kt, kl, 1);
+            dequant_half(cur.vc[0], cur.vc[1], cur.vs.x, vt, kl, 0);
+            dequant_half(cur.vc[2], cur.vc[3], cur.vs.y, vt, kl, 1);
+            fence_async_smem();
+            mbar_arrive(smem_u32(&sh.kv_full[st]));
+            cur = nxt;
+        }
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ MMA issue (warp 8)
+        constexpr uint32_t idesc_qk = umma_idesc_f16(false, 64);
+        constexpr uint32_t idesc_pv = umma_idesc_f16(true, 128);
+        const uint32_t kt_addr = smem_u32(Kt), vt_addr = smem_u32(Vt);
+        bool ok = wait_or_abort(smem_u32(&sh.q_ready[0]), 0u, abort, a.ctl, 40u, 0) &&
+                  wait_or_abort(smem_u32(&sh.q_ready[1]), 0u, abort, a.ctl, 41u, 0);
+        // Descriptors of stage 0; a stage or k-step offset is added to the
+        // start-address field (bits 0..13, address >> 4): shared-memory
+        // addresses stay below 256 KB, so the field never carries.
+        const uint64_t kdesc0 = umma_desc(kt_addr, 16, 1024);
+        const uint64_t vdesc0 = umma_desc(vt_addr, 8192, 1024);
+        auto issue_qk = [&](int qi, int st) {
+            const uint64_t d0 = kdesc0 + (uint64_t)((st * kStageBytes) >> 4);
+            const uint32_t dt = tmem + kColS + 64u * qi;
+            const uint32_t at = tmem + kColQ + 64u * qi;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ts(dt, at + (uint32_t)(ks * 8),
+                       d0 + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), idesc_qk,
+                       ks > 0 ? 1u : 0u);
+            mma_commit(smem_u32(&sh.s_full[qi]));
+        };
+        auto issue_pv = [&](int qi, int st, bool first) {
+            const uint64_t d0 = vdesc0 + (uint64_t)((st * kStageBytes) >> 4);
+            const uint32_t dt = tmem + kColO + 128u * qi;
+            const uint32_t at = tmem + kColS + 64u * qi;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ts(dt, at + (uint32_t)(ks * 8), d0 + (uint64_t)((ks * 2048) >> 4), idesc_pv,
+                       (ks > 0 || !first) ? 1u : 0u);
+        };
+        if (ok) {
+            tc_fence_after();
+            ok = wait_or_abort(smem_u32(&sh.kv_full[0]), 0u, abort, a.ctl, 42u, 0);
+            if (ok) {
+                tc_fence_after();
+                issue_qk(0, 0);
+                issue_qk(1, 0);
+            }
+        }
+        for (int t = 0; t < ntiles && ok; ++t) {
+            const int st = t % kStages;
+            ok = wait_or_abort(smem_u32(&sh.p_full[0]), (uint32_t)(t & 1), abort, a.ctl, 43u, t);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(0, st, t == 0);
+            const bool more = t + 1 < ntiles;
+            const int st2 = (t + 1) % kStages;
+            if (more) {
+                ok = wait_or_abort(smem_u32(&sh.kv_full[st2]), (uint32_t)(((t + 1) / kStages) & 1),
+                                   abort, a.ctl, 44u, t + 1);
+                if (!ok) break;
+                tc_fence_after();
+                issue_qk(0, st2);
+            }
+            ok = wait_or_abort(smem_u32(&sh.p_full[1]), (uint32_t)(t & 1), abort, a.ctl, 45u, t);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(1, st, t == 0);
+            mma_commit(smem_u32(&sh.kv_empty[st]));
+            if (more) issue_qk(1, st2);
+        }
+        if (ok) mma_commit(smem_u32(&sh.o_final));
+        // every MMA of this thread is complete before tensor memory is freed
+        mma_commit(smem_u32(&sh.drain));
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(smem_u32(&sh.drain), 0u) && globaltimer_ns() - t0 < kWaitLimitNs)
+            __nanosleep(64);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kColsW));
+    }
+}
+
+}  // namespace
+
+nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                   int H, const void* Q, int T_q, void* O, int o_dtype,
+                                   float softmax_scale, void* ws, cudaStream_t stream) {
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(attention_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemW) != cudaSuccess)
+            return NVFP4KV_ERR_CUDA;
+        configured = true;
+    }
+    WsArgs a;
+    for (int i = 0; i < n_chunks; ++i) {
+        a.chunk[i].k_codes = chunks[i].k_codes;
+        a.chunk[i].k_scales = chunks[i].k_scales;
+        a.chunk[i].v_codes = chunks[i].v_codes;
+        a.chunk[i].v_scales = chunks[i].v_scales;
+        a.chunk[i].k_mean = chunks[i].k_mean;
+        a.chunk[i].tensor_scales = chunks[i].tensor_scales;
+    }
+    a.n_chunks = n_chunks;
+    a.T_c = T_c;
+    a.H = H;
+    a.T_q = T_q;
+    a.Q = static_cast<const uint16_t*>(Q);
+    a.O = O;
+    a.o_f32 = o_dtype == NVFP4KV_F32 ? 1 : 0;
+    a.scale_log2 = softmax_scale * kLog2eW;
+    a.ctl = static_cast<Control*>(ws);
+    dim3 grid((T_q + 255) / 256, H);
+    attention_ws_kernel<<<grid, kThreadsW, kSmemW, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+}  // namespace nvfp4kv

@@ -55,8 +55,13 @@ nvfp4kv_status launch_attention_tc(const nvfp4kv_chunk_view* chunks, int n_chunk
                                    int H, const void* Q, int T_q, void* O, int o_dtype,
                                    float softmax_scale, void* ws, cudaStream_t stream);
 
-// Sink-window attention: the tcgen05 kernel, or the mma.sync kernel when the
-// environment variable NVFP4KV_ATTENTION_KERNEL=mma selects it (cross-checks).
+nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                   int H, const void* Q, int T_q, void* O, int o_dtype,
+                                   float softmax_scale, void* ws, cudaStream_t stream);
+
+// Sink-window attention: the warp-specialized tcgen05 kernel; the environment
+// variable NVFP4KV_ATTENTION_KERNEL selects the single-group tcgen05 kernel
+// ("tc1") or the mma.sync kernel ("mma") instead, for cross-checks.
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                 int H, const void* Q, int T_q, void* O, int o_dtype,
                                 float softmax_scale, void* ws, cudaStream_t stream);
