@@ -23,6 +23,7 @@ O inside the timed region).
 independent replicas (no collective on the data path), weak scaling.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -44,6 +45,27 @@ WORKLOAD = ("one layer step: NVFP4-quantize K,V [7040,24,128] bf16 into the cach
             "sink-window attention Q [7040,24,128] over S_g=1, S_s=1, W=3 chunks (35,200 keys)")
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture of the layer step (summaries under profiles/), valid only for the kernel
+# source it was taken on: a changed source reports null until it is captured again.
+NCU_TRAFFIC = {
+    "attention": ("sink_window_video_b200/csrc/attention_ws.cu",
+                  "7c92672a848293abc612987a15e780aa6d40d7dbf4c805bc1b65ef10239375fb", 194599168),
+    "quantize": ("sink_window_video_b200/csrc/quant.cu",
+                 "9e3baa03cec1462f4f474203a0edd716f6f142c9c535cce06c4e93141d5594d2", 133928960),
+}
+
+
+def ncu_traffic(which):
+    path, sha, nbytes = NCU_TRAFFIC[which]
+    try:
+        with open(os.path.join(ROOT, path), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return nbytes if digest == sha else None
 
 
 def keys_per_step():
@@ -386,11 +408,12 @@ def main():
                        "l2": "inputs rotate over 4 sets of K,V,Q (520 MB) > 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": "sink_window_attention",
                          "achieved": attn_tf, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": attn_tf / tpeak, "traffic": None,
+                         "frac": attn_tf / tpeak, "traffic": ncu_traffic("attention"),
                          "peak_source": f"{peak_src} bf16 sustained"},
             "quantize": {"kernel": "nvfp4kv_quantize_chunk", "bound": "hbm",
                          "achieved": quant_gbs, "peak": hpeak, "unit": "GB/s",
                          "frac": quant_gbs / hpeak, "bytes_per_launch": quant_bytes(),
+                         "traffic": ncu_traffic("quantize"),
                          "ms_per_launch": r["ms_quant"], "peak_source": f"{peak_src} hbm"},
             "attention": {"ms_per_launch": r["ms_attn"], "flops_per_launch": attn_flops(),
                           "tflops": attn_tf},
