@@ -255,29 +255,124 @@ def run_ours(args, rank, world, local):
         raise RuntimeError("device status not OK after the timed steps")
     ms_total = max_over_ranks(ms_total, world)
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step copies
+    # its K, V, Q from pinned host memory and reads its O back; the copies run
+    # on two copy streams into double buffers, so step i+1's inputs and step
+    # i-1's output cross the host link while step i computes
     e2e_ms = None
     if not args.no_e2e:
-        O_host = torch.empty((T, H, d), dtype=torch.bfloat16).pin_memory()
+        up = torch.cuda.Stream(device=dev)        # host -> device (its own copy engine)
+        down = torch.cuda.Stream(device=dev)      # device -> host
+        dbuf = [tuple(torch.empty_like(x) for x in pool[0]) for _ in range(2)]
+        obuf = [torch.empty_like(O) for _ in range(2)]
+        O_host = [torch.empty((T, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        loaded = [torch.cuda.Event() for _ in range(2)]
+        consumed = [torch.cuda.Event() for _ in range(2)]
+        drained = [torch.cuda.Event() for _ in range(2)]
+        n_e2e = args.e2e_steps
+
+        def upload(i):
+            b = i % 2
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(consumed[b])          # step i-2 no longer reads this buffer
+                for dst, src in zip(dbuf[b], pinned[i % CFG["pool"]]):
+                    dst.copy_(src, non_blocking=True)
+                loaded[b].record(up)
+
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(args.e2e_steps):
-            Kh, Vh, Qh = pinned[i % CFG["pool"]]
-            K = Kh.to(dev, non_blocking=True)
-            V = Vh.to(dev, non_blocking=True)
-            Q = Qh.to(dev, non_blocking=True)
+        upload(0)
+        for i in range(n_e2e):
+            b = i % 2
+            if i + 1 < n_e2e:
+                upload(i + 1)
+            stream.wait_event(loaded[b])
+            if i >= 2:
+                stream.wait_event(drained[b])            # step i-2's O has left obuf[b]
+            K, V, Q = dbuf[b]
             cache.append(0, K, V)
-            cache.attention(0, Q, O)
-            O_host.copy_(O, non_blocking=True)
+            cache.attention(0, Q, obuf[b])
+            consumed[b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(consumed[b])
+                O_host[b].copy_(obuf[b], non_blocking=True)
+                drained[b].record(down)
+        stream.wait_stream(down)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
+
+    rollouts = None
+    if not args.no_rollout:
+        rollouts = [run_rollout(swv, cfg, pool, O, stream, world) for cfg in ROLLOUTS]
 
     return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
-                e2e_ms=e2e_ms)
+                e2e_ms=e2e_ms, rollouts=rollouts)
+
+
+# ------------------------------------------------------------------ rollouts
+
+ROLLOUTS = (synth.ROLLOUT, synth.MULTISHOT)
+
+
+def rollout_keyset_sizes(swv, cfg):
+    """Chunks attended at each step of the schedule (the same in every layer),
+    from the cache's own bookkeeping (advance + keyset, no device work)."""
+    c = swv.KVCache(1, CFG["H"], CFG["T_c"], cfg["S_g"], cfg["S_s"], cfg["W"])
+    sizes = []
+    for n in range(cfg["chunks"]):
+        if n in cfg["switches"]:
+            c.rebind_shot_sink(n)
+        c.advance(0)
+        sizes.append(len(c.keyset(0)))
+    return sizes
+
+
+def run_rollout(swv, cfg, pool, O, stream, world):
+    """One streaming rollout: every chunk of the schedule through every layer
+    (quantize into the cache, then sink-window attention), shot switches
+    re-binding A_s; inputs rotate over the device-resident pool."""
+    import torch
+    T, H = CFG["T_c"], CFG["H"]
+    layers, chunks = cfg["layers"], cfg["chunks"]
+    sizes = rollout_keyset_sizes(swv, cfg)
+    flops = sum(sizes) * layers * attn_flops(T_q=T, L=T)
+    n_quant = chunks * layers
+    cache = swv.KVCache(layers, H, T, cfg["S_g"], cfg["S_s"], cfg["W"])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for n in range(chunks):
+        if n in cfg["switches"]:
+            cache.rebind_shot_sink(n)
+        for layer in range(layers):
+            K, V, Q = pool[(n * layers + layer) % len(pool)]
+            cache.append(layer, K, V)
+            cache.attention(layer, Q, O)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if cache.check_status() != swv.OK:
+        raise RuntimeError("device status not OK after the rollout")
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    del cache
+    peaks, src = load_peaks()
+    tpeak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    t_roof = flops / (tpeak * 1e12) + n_quant * quant_bytes() / (hpeak * 1e9)
+    value = chunks * world / (ms / 1e3)
+    return {"workload": (f"{cfg['name']}: {chunks} chunks x {layers} layers of [{T},{H},128], "
+                         f"S_g={cfg['S_g']}, S_s={cfg['S_s']}, W={cfg['W']}, shot switches at "
+                         f"{list(cfg['switches']) or 'none'}"),
+            "chunks_per_s": value, "ms": ms, "attention_flops": flops,
+            "gpu_launches": 2 * n_quant,
+            "quantizations": n_quant, "keyset_sizes": sizes,
+            "roofline_chunks_per_s": chunks * world / t_roof, "frac": value * t_roof / (chunks * world),
+            "roofline_basis": f"{src} bf16 sustained + {src} hbm, attention and quantizer serial"}
 
 
 # ------------------------------------------------------------------ oracle (CPU)
@@ -378,6 +473,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rollout", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -425,6 +521,8 @@ def main():
             line["e2e"] = {"value": attn_flops() * world / (r["e2e_ms"] / 1e3) / 1e12,
                            "unit": "TFLOP/s", "h2d_bytes_per_step": 3 * n * 2,
                            "d2h_bytes_per_step": n * 2, "ms_per_step": r["e2e_ms"]}
+        if r["rollouts"] is not None:
+            line["rollouts"] = r["rollouts"]
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = OracleSample(rows=args.ref_rows).baseline()
         print(json.dumps(line))

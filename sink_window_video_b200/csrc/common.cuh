@@ -30,7 +30,9 @@ struct Control {
     unsigned bar_count;   // grid barrier: CTAs arrived at the current barrier
     unsigned bar_gen;     // grid barrier: generation, bumped by the last arrival
     unsigned diag[4];     // first wait that gave up: site, block (x | y << 16), step, phase
-    unsigned pad[57];
+    unsigned pad0[2];
+    unsigned long long stamp[8];   // %globaltimer at CTA 0's phase boundaries (diagnostics)
+    unsigned pad[38];
 };
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -85,7 +87,7 @@ __device__ __forceinline__ bool grid_barrier(Control* ctl) {
                     ok = 0;
                     break;
                 }
-                __nanosleep(100);
+                __nanosleep(32);
             }
         }
         __threadfence();

@@ -8,19 +8,26 @@
 // lower squared error kept; K has its per-head, per-channel mean over the
 // chunk's tokens removed first and kept in fp32.
 //
-// One cooperative persistent kernel per chunk, three phases split by grid
-// barriers:
-//   1. stats:    every (64-token segment, 256-column group) of K gives column
-//                sums (fp32, in token order), column min and max (bf16, exact);
-//                V gives per-CTA max |V|.  One 128-bit load per lane per token.
-//   2. finalize: per column, the segment sums are added in segment order and
-//                divided by T (the mean); max |K - mean| comes from the column
-//                min/max (x -> RN(x - mean) is monotone), reduced per CTA.
-//   3. encode:   two lanes per 16-element block (8 elements each, one 128-bit
-//                load); the block max and the two half-errors meet through one
-//                shuffle each; each lane of a pair computes one target's block
-//                scale and swaps it with its partner; codes are stored packed,
-//                head-major, 4 bytes per lane.
+// One cooperative persistent kernel per chunk, four phases split by grid
+// barriers.  HBM is read once (K and V, 2 bytes per element); the second
+// read of each tensor hits L2 (126 MB holds both), steered by L2 eviction
+// hints:
+//   A. max |V|:  one streaming pass over V, per-CTA partial maxima.
+//   B. the K column statistics of every (64-token segment, 256-column group)
+//      -- fp32 column sums in token order, bf16 column min and max -- read
+//      from HBM, and the encoding of V (its tensor scale is known after A)
+//      from L2: every warp takes its statistics units first and its V units
+//      after, so each SM interleaves K's HBM stream with V's arithmetic.
+//   C. per column: the segment sums added in segment order and divided by
+//      T (the mean); max |K - mean| from the column min/max (x -> RN(x - mean)
+//      is monotone).
+//   D. the encoding of K from L2.
+// Encoding: two lanes per 16-element block (8 elements each, one 128-bit
+// load); the block max and the two half-errors meet through one shuffle each.
+// Both targets' block scales come from one paired division, their decoded
+// step D and RN(1/D) from a 256-entry table per tensor, and every division
+// x / D is Markstein's correctly rounded quotient (one multiply, two fused
+// multiply-adds) on float pairs.
 // Every fp32 step that the definition fixes is one IEEE operation (explicit
 // _rn intrinsics, compiled without FMA contraction), so codes, scales, means
 // and tensor scales are bit-identical to the definition.
@@ -30,8 +37,16 @@
 namespace nvfp4kv {
 namespace {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 768;       // one CTA per SM: 24 warps
 constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kEncTokens = 8;          // tokens per encoding unit (one warp)
+constexpr int kFinCols = 32;           // columns per finalize block (one per lane)
+constexpr int kFinSegs = 120;          // segments staged per finalize pass (5 per warp)
+// Markstein's quotient is correctly rounded when no step underflows: the
+// tensor scale and the block max are kept above these bounds, else the
+// quotient is an IEEE division.
+constexpr float kFastMinScale = 0x1p-90f;
+constexpr float kFastMinBlockMax = 0x1p-100f;
 
 struct QuantArgs {
     const uint4* K;
@@ -49,6 +64,17 @@ struct QuantArgs {
     float* kpart;
     float* vpart;
     Control* ctl;
+    float one;              // 1 as a run-time value (see encode8_fast)
+};
+
+struct QuantShared {
+    float red[kQuantWarps];
+    unsigned qhead;                           // this CTA's phase-B work queue
+    float2 tab[256];                          // per E4M3 code: D = RN(code * s), RN(1/D)
+    uint8_t sb[kQuantWarps][kEncTokens * 8];  // staged scale bytes of one unit per warp
+    float fsum[kFinSegs][kFinCols];           // finalize staging
+    unsigned short fmin[kFinSegs][kFinCols];
+    unsigned short fmax[kFinSegs][kFinCols];
 };
 
 __device__ __forceinline__ float block_max(float v, float* red) {
@@ -70,7 +96,74 @@ __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// ---------------------------------------------------------------- phase 1
+// L2 eviction policies: inputs read twice are kept (evict_last) on the first
+// read and released (evict_first) on the second.
+__device__ __forceinline__ uint64_t policy_keep() {
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_release() {
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint4 ld_hint(const uint4* p, uint64_t pol) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p), "l"(pol));
+    return r;
+}
+
+// The tensor scale from the per-CTA partial maxima, and the decode table.
+__device__ __forceinline__ float tensor_scale_and_table(const float* part, QuantShared& sh) {
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < gridDim.x; i += blockDim.x) m = fmaxf(m, __ldcg(part + i));
+    const float A = block_max(m, sh.red);
+    const float s = A > 0.0f ? __fdiv_rn(A, kTensorScaleDiv) : 1.0f;
+    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+        const float D = __fmul_rn(e4m3_to_f32((uint32_t)c), s);
+        sh.tab[c] = make_float2(D, D > 0.0f ? __frcp_rn(D) : 0.0f);
+    }
+    __syncthreads();
+    return s;
+}
+
+// ---------------------------------------------------------------- phase A
+
+__device__ void phase_vmax(const QuantArgs& a, QuantShared& sh, uint64_t keep) {
+    const size_t n16 = (size_t)a.T * a.HD / 8;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t m = 0;                               // two bf16 magnitudes, lane-wise max
+    for (; i + 15 * stride < n16; i += 16 * stride) {
+        uint4 w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) w[k] = ld_hint(a.V + i + k * stride, keep);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            m = __vmaxu2(m, w[k].x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w[k].y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w[k].z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w[k].w & 0x7FFF7FFFu);
+        }
+    }
+    for (; i < n16; i += stride) {
+        const uint4 w = ld_hint(a.V + i, keep);
+        m = __vmaxu2(m, w.x & 0x7FFF7FFFu);
+        m = __vmaxu2(m, w.y & 0x7FFF7FFFu);
+        m = __vmaxu2(m, w.z & 0x7FFF7FFFu);
+        m = __vmaxu2(m, w.w & 0x7FFF7FFFu);
+    }
+    const float v = fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+    const float b = block_max(v, sh.red);
+    if (threadIdx.x == 0) {
+        a.vpart[blockIdx.x] = b;
+    }
+}
+
+// ---------------------------------------------------------------- K column statistics
 
 __device__ __forceinline__ void stats_k_token(const uint4& w, float* sum, uint32_t* mn,
                                               uint32_t* mx) {
@@ -86,232 +179,404 @@ __device__ __forceinline__ void stats_k_token(const uint4& w, float* sum, uint32
     }
 }
 
-__device__ __forceinline__ void stats_v_token(const uint4& w, uint32_t* mx) {
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) mx[j] = as_u32(__hmax2(as_bf162(mx[j]), as_bf162(u[j] & 0x7FFF7FFFu)));
-}
-
-__device__ void phase_stats(const QuantArgs& a, float* red) {
+// One (64-token segment, 256-column group) of K: lane = 8 columns.
+__device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
     const int lane = threadIdx.x & 31;
-    const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
-    const int nw = gridDim.x * kQuantWarps;
-    const int upt = a.nseg * a.ngroups;
+    const int s = unit / a.ngroups;
+    const int g = unit - s * a.ngroups;
+    const int col = g * 256 + lane * 8;
+    if (col >= a.HD) return;
+    const int t0 = s * kSegment;
+    const int nt = min(kSegment, a.T - t0);
     const size_t row8 = (size_t)a.HD / 8;
-    float vmax = 0.0f;
-    for (int u = wg; u < 2 * upt; u += nw) {
-        const bool isK = u < upt;
-        const int uu = isK ? u : u - upt;
-        const int s = uu / a.ngroups;
-        const int g = uu - s * a.ngroups;
-        const int col = g * 256 + lane * 8;
-        if (col >= a.HD) continue;
-        const int t0 = s * kSegment;
-        const int nt = min(kSegment, a.T - t0);
-        const uint4* src = (isK ? a.K : a.V) + (size_t)t0 * row8 + col / 8;
-        if (isK) {
-            float sum[8];
-            uint32_t mn[4], mx[4];
+    const uint4* src = a.K + (size_t)t0 * row8 + col / 8;
+    float sum[8];
+    uint32_t mn[4], mx[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
+    for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) { mn[j] = 0x7F807F80u; mx[j] = 0xFF80FF80u; }
-            int t = 0;
-            for (; t + 8 <= nt; t += 8) {
-                uint4 w[8];
+    for (int j = 0; j < 4; ++j) { mn[j] = 0x7F807F80u; mx[j] = 0xFF80FF80u; }
+    int t = 0;
+    for (; t + 16 <= nt; t += 16) {
+        uint4 w[16];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) w[k] = ld_stream(src + (size_t)(t + k) * row8);
+        for (int k = 0; k < 16; ++k) w[k] = ld_hint(src + (size_t)(t + k) * row8, keep);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) stats_k_token(w[k], sum, mn, mx);
-            }
-            for (; t < nt; ++t) stats_k_token(ld_stream(src + (size_t)t * row8), sum, mn, mx);
-            float4* ps = reinterpret_cast<float4*>(a.psum + (size_t)s * a.HD + col);
-            ps[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
-            ps[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
-            const size_t w2 = ((size_t)s * a.HD + col) / 2;
-            *reinterpret_cast<uint4*>(a.pmin + w2) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
-            *reinterpret_cast<uint4*>(a.pmax + w2) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
-        } else {
-            uint32_t mx[4] = {0u, 0u, 0u, 0u};
-            int t = 0;
-            for (; t + 8 <= nt; t += 8) {
-                uint4 w[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) w[k] = ld_stream(src + (size_t)(t + k) * row8);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) stats_v_token(w[k], mx);
-            }
-            for (; t < nt; ++t) stats_v_token(ld_stream(src + (size_t)t * row8), mx);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                vmax = fmaxf(vmax, __uint_as_float(mx[j] << 16));
-                vmax = fmaxf(vmax, __uint_as_float(mx[j] & 0xFFFF0000u));
-            }
-        }
+        for (int k = 0; k < 16; ++k) stats_k_token(w[k], sum, mn, mx);
     }
-    const float b = block_max(vmax, red);
-    if (threadIdx.x == 0) a.vpart[blockIdx.x] = b;
+    for (; t < nt; ++t) stats_k_token(ld_hint(src + (size_t)t * row8, keep), sum, mn, mx);
+    float4* ps = reinterpret_cast<float4*>(a.psum + (size_t)s * a.HD + col);
+    ps[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+    ps[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
+    const size_t w2 = ((size_t)s * a.HD + col) / 2;
+    *reinterpret_cast<uint4*>(a.pmin + w2) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
+    *reinterpret_cast<uint4*>(a.pmax + w2) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
 }
 
-// ---------------------------------------------------------------- phase 2
+// ---------------------------------------------------------------- encoding
 
-__device__ void phase_finalize(const QuantArgs& a, float* red) {
-    float kp = 0.0f;
-    const int stride = gridDim.x * blockDim.x;
-    const float Tf = (float)a.T;
-    const unsigned short* pmin = reinterpret_cast<const unsigned short*>(a.pmin);
-    const unsigned short* pmax = reinterpret_cast<const unsigned short*>(a.pmax);
-    for (int col = blockIdx.x * blockDim.x + threadIdx.x; col < a.HD; col += stride) {
-        float S = 0.0f, mn = INFINITY, mx = -INFINITY;
-        int s = 0;
-        for (; s + 8 <= a.nseg; s += 8) {
-            float p[8];
-            unsigned short n[8], x[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const size_t i = (size_t)(s + k) * a.HD + col;
-                p[k] = __ldcg(a.psum + i);
-                n[k] = __ldcg(pmin + i);
-                x[k] = __ldcg(pmax + i);
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                S = __fadd_rn(S, p[k]);
-                mn = fminf(mn, __uint_as_float((uint32_t)n[k] << 16));
-                mx = fmaxf(mx, __uint_as_float((uint32_t)x[k] << 16));
-            }
-        }
-        for (; s < a.nseg; ++s) {
-            const size_t i = (size_t)s * a.HD + col;
-            S = __fadd_rn(S, __ldcg(a.psum + i));
-            mn = fminf(mn, __uint_as_float((uint32_t)__ldcg(pmin + i) << 16));
-            mx = fmaxf(mx, __uint_as_float((uint32_t)__ldcg(pmax + i) << 16));
-        }
-        const float mu = __fdiv_rn(S, Tf);
-        a.k_mean[col] = mu;
-        kp = fmaxf(kp, fmaxf(fabsf(__fsub_rn(mx, mu)), fabsf(__fsub_rn(mn, mu))));
-    }
-    const float b = block_max(kp, red);
-    if (threadIdx.x == 0) a.kpart[blockIdx.x] = b;
+__device__ __forceinline__ float max_abs8(const float2* x) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(x[0].x)), "f"(fabsf(x[0].y)), "f"(fabsf(x[1].x)));
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(d), "f"(fabsf(x[1].y)), "f"(fabsf(x[2].x)));
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(d), "f"(fabsf(x[2].y)), "f"(fabsf(x[3].x)));
+    return fmaxf(d, fabsf(x[3].y));
 }
 
-// ---------------------------------------------------------------- phase 3
+// f16 -> f32 (exact) as a mixed-precision add of -0: a full-rate FMA-pipe
+// operation, where cvt.f32.f16 issues at half rate.
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h2) {
+    float lo, hi;
+    asm("{.reg .b16 l, h;\n"
+        "mov.b32 {l, h}, %2;\n"
+        "add.rn.f32.f16 %0, l, 0f80000000;\n"
+        "add.rn.f32.f16 %1, h, 0f80000000;}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h2));
+    return make_float2(lo, hi);
+}
 
-// Eight elements x against one candidate (block step D, its reciprocal r):
+// Four fp32 pairs -> the packed E2M1 codes (byte j = elements 2j, 2j+1) and
+// their decoded values as four f16x2, from the same conversion bytes.
+__device__ __forceinline__ uint32_t cvt_e2m1x8_dec(const float* v, uint32_t* h) {
+    uint32_t r;
+    asm("{\n"
+        ".reg .b8 b0, b1, b2, b3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n"
+        "cvt.rn.f16x2.e2m1x2 %1, b0;\n"
+        "cvt.rn.f16x2.e2m1x2 %2, b1;\n"
+        "cvt.rn.f16x2.e2m1x2 %3, b2;\n"
+        "cvt.rn.f16x2.e2m1x2 %4, b3;\n"
+        "mov.b32 %0, {b0, b1, b2, b3};\n"
+        "}"
+        : "=r"(r), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+          "f"(v[7]));
+    return r;
+}
+
+// Eight elements (four pairs) against one candidate step D with r = RN(1/D):
 // packed codes q (byte j = elements 2j, 2j+1) and the sequential sum of the
-// eight squared errors (x - decode(q) * D)^2.
-__device__ __forceinline__ void encode_half(const float* x, float D, float r, uint32_t& q,
-                                            float& err) {
+// eight squared errors RN(RN(x - RN(decode(q) * D))^2).
+// The quotient is Markstein's, computed for -x / D so that a zero keeps its
+// sign: n0 = RN(x (-r)), e = x + n0 D (exact), n1 = RN(n0 - e r) = -RN(x / D).
+// The codes of -x / D are those of x / D with the sign bits flipped (one XOR
+// for the stored word); their decoded values dq' = -dq give the error
+// directly: RN(x - RN(dq D)) = RN(x + RN(dq' D)).
+// The compiler merges a paired product followed by a paired sum into one
+// fused multiply-add, which would skip the product's rounding; every sum is
+// therefore written as a fused multiply-add whose other factor is 1 held in a
+// run-time value (exact, and not mergeable).
+__device__ __forceinline__ void encode8_fast(const float2* x, float2 Dr, float one, uint32_t& q,
+                                             float& err) {
+    const float2 NR = make_float2(-Dr.y, -Dr.y);
+    const float2 D2 = make_float2(Dr.x, Dr.x);
     float y[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = div_markstein(x[i], D, r);
-    q = D > 0.0f ? cvt_e2m1x8(y) : 0u;
+    for (int j = 0; j < 4; ++j) {
+        const float2 n0 = __fmul2_rn(x[j], NR);
+        const float2 e = __ffma2_rn(n0, D2, x[j]);
+        const float2 n1 = __ffma2_rn(e, NR, n0);
+        y[2 * j] = n1.x;
+        y[2 * j + 1] = n1.y;
+    }
     uint32_t h[4];
-    cvt_e2m1x8_to_f16x2(q, h);
+    q = cvt_e2m1x8_dec(y, h) ^ 0x88888888u;
+    const float2 ONE = make_float2(one, one);
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 p = __fmul2_rn(f16x2_to_f32x2(h[j]), D2);      // RN(dq' D) = -RN(dq D)
+        const float2 d = __ffma2_rn(p, ONE, x[j]);                   // RN(x - RN(dq D))
+        const float2 sq = __fmul2_rn(d, d);
+        acc = (j == 0) ? sq.x : __fmaf_rn(sq.x, one, acc);
+        acc = __fmaf_rn(sq.y, one, acc);
+    }
+    err = acc;
+}
+
+// The same with IEEE divisions (tensor scales too small for the fast path);
+// out of line, so the rare path costs no instruction-cache space in the loop.
+struct Enc8 {
+    uint32_t q;
+    float err;
+};
+
+__device__ __noinline__ Enc8 encode8_slow(float x0, float x1, float x2, float x3, float x4,
+                                          float x5, float x6, float x7, float D) {
+    const float x[8] = {x0, x1, x2, x3, x4, x5, x6, x7};
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = D > 0.0f ? __fdiv_rn(x[i], D) : 0.0f;
+    Enc8 r;
+    r.q = cvt_e2m1x8(y);
+    uint32_t h[4];
+    cvt_e2m1x8_to_f16x2(r.q, h);
     float acc = 0.0f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const float e0 = __fsub_rn(x[2 * j], __fmul_rn(f16lo(h[j]), D));
         const float e1 = __fsub_rn(x[2 * j + 1], __fmul_rn(f16hi(h[j]), D));
-        const float s0 = __fmul_rn(e0, e0);
-        const float s1 = __fmul_rn(e1, e1);
-        acc = (j == 0) ? s0 : __fadd_rn(acc, s0);
-        acc = __fadd_rn(acc, s1);
+        acc = (j == 0) ? __fmul_rn(e0, e0) : __fadd_rn(acc, __fmul_rn(e0, e0));
+        acc = __fadd_rn(acc, __fmul_rn(e1, e1));
     }
-    err = acc;
+    r.err = acc;
+    return r;
 }
 
-__device__ void phase_encode(const QuantArgs& a, float* red) {
-    float kp = 0.0f, vp = 0.0f;
-    for (int i = threadIdx.x; i < gridDim.x; i += blockDim.x) {
-        kp = fmaxf(kp, __ldcg(a.kpart + i));
-        vp = fmaxf(vp, __ldcg(a.vpart + i));
-    }
-    const float AK = block_max(kp, red);
-    const float AV = block_max(vp, red);
-    const float sK = AK > 0.0f ? __fdiv_rn(AK, kTensorScaleDiv) : 1.0f;
-    const float sV = AV > 0.0f ? __fdiv_rn(AV, kTensorScaleDiv) : 1.0f;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        a.tensor_scales[0] = sK;
-        a.tensor_scales[1] = sV;
-    }
+__device__ __noinline__ float2 ratio_slow(float ab, float ms6, float ms4) {
+    return make_float2(__fdiv_rn(ab, ms6), __fdiv_rn(ab, ms4));
+}
 
+// One unit: head h, tokens [t0, t0 + 8) of K (mean subtracted) or V (mean
+// -0: x + (-0) = x exactly, signed zeros included).  Lane = (token parity,
+// 8-channel group); iteration it covers tokens t0 + 2 it + {0, 1}, with the
+// next iteration's 16 bytes loaded ahead.
+__device__ void encode_unit(const QuantArgs& a, QuantShared& sh, bool isK, int h, int t0,
+                            float s, bool fast, float ms6, float ms4, float2 rm,
+                            uint64_t release) {
     const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int c8 = lane & 15;                 // 8-channel group of this lane
+    const int tsub = lane >> 4;
+    const bool odd = (lane & 1) != 0;         // second half of its 16-block
+    const uint4* src = isK ? a.K : a.V;
+    float2 nmu[4];
+    if (isK) {
+        const float4* mp = reinterpret_cast<const float4*>(a.k_mean + h * kHeadDim + c8 * 8);
+        const float4 m0 = __ldcg(mp), m1 = __ldcg(mp + 1);
+        nmu[0] = make_float2(-m0.x, -m0.y);
+        nmu[1] = make_float2(-m0.z, -m0.w);
+        nmu[2] = make_float2(-m1.x, -m1.y);
+        nmu[3] = make_float2(-m1.z, -m1.w);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) nmu[j] = make_float2(-0.0f, -0.0f);
+    }
+    uint32_t* codes = reinterpret_cast<uint32_t*>(isK ? a.k_codes : a.v_codes);
+    auto load = [&](int it) {
+        const int t = t0 + 2 * it + tsub;
+        return t < a.T ? ld_hint(src + ((size_t)t * a.H + h) * 16 + c8, release)
+                       : make_uint4(0u, 0u, 0u, 0u);
+    };
+    uint4 wn = load(0);
+#pragma unroll 1
+    for (int it = 0; it < kEncTokens / 2; ++it) {
+        const uint4 w = wn;
+        if (it + 1 < kEncTokens / 2) wn = load(it + 1);
+        const int t = t0 + 2 * it + tsub;
+        float2 x[4];
+        {
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                x[j] = __fadd2_rn(make_float2(__uint_as_float(u[j] << 16),
+                                              __uint_as_float(u[j] & 0xFFFF0000u)),
+                                  nmu[j]);                          // RN(K - mean), or V
+        }
+        const float ah = max_abs8(x);
+        const float ab = fmaxf(ah, __shfl_xor_sync(0xFFFFFFFFu, ah, 1));
+        // block scales of both targets: RN(ab / RN(6 s)), RN(ab / RN(4 s))
+        float2 rat;
+        if (fast && ab >= kFastMinBlockMax) {
+            const float2 AB = make_float2(ab, ab);
+            const float2 q0 = __fmul2_rn(AB, rm);
+            const float2 e = __ffma2_rn(q0, make_float2(-ms6, -ms4), AB);
+            rat = __ffma2_rn(e, rm, q0);
+        } else {
+            rat = ratio_slow(ab, ms6, ms4);
+        }
+        const uint32_t sbp = cvt_e4m3x2(rat.x, rat.y);
+        const uint32_t sb6 = sbp & 0xFFu, sb4 = sbp >> 8;
+        const float2 t6 = sh.tab[sb6], t4 = sh.tab[sb4];
+        uint32_t q6, q4;
+        float e6, e4;
+        if (fast) {
+            encode8_fast(x, t6, a.one, q6, e6);
+            encode8_fast(x, t4, a.one, q4, e4);
+        } else {
+            const Enc8 r6 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y,
+                                         x[3].x, x[3].y, t6.x);
+            const Enc8 r4 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y,
+                                         x[3].x, x[3].y, t4.x);
+            q6 = r6.q; e6 = r6.err;
+            q4 = r4.q; e4 = r4.err;
+        }
+        // block error = (elements 0..7) + (elements 8..15)
+        const float E6 = __fadd_rn(e6, __shfl_xor_sync(0xFFFFFFFFu, e6, 1));
+        const float E4 = __fadd_rn(e4, __shfl_xor_sync(0xFFFFFFFFu, e4, 1));
+        const bool keep4 = E4 < E6;
+        uint32_t q = keep4 ? q4 : q6;
+        if (!((keep4 ? t4.x : t6.x) > 0.0f)) q = 0u;      // a zero step stores +0 codes
+        if (t < a.T) codes[((size_t)h * a.T + t) * 16 + c8] = q;
+        if (!odd) sh.sb[warp][(2 * it + tsub) * 8 + (c8 >> 1)] = (uint8_t)(keep4 ? sb4 : sb6);
+    }
+    __syncwarp();
+    if (lane < kEncTokens && t0 + lane < a.T) {
+        uint8_t* scales = isK ? a.k_scales : a.v_scales;
+        *reinterpret_cast<uint2*>(scales + ((size_t)h * a.T + t0 + lane) * 8) =
+            *reinterpret_cast<const uint2*>(&sh.sb[warp][lane * 8]);
+    }
+    __syncwarp();
+}
+
+struct EncodeConsts {
+    float s, ms6, ms4;
+    float2 rm;
+    bool fast;
+};
+
+__device__ __forceinline__ EncodeConsts encode_consts(float s) {
+    EncodeConsts c;
+    c.s = s;
+    c.ms6 = __fmul_rn(6.0f, s);
+    c.ms4 = __fmul_rn(4.0f, s);
+    c.rm = make_float2(__frcp_rn(c.ms6), __frcp_rn(c.ms4));
+    c.fast = s >= kFastMinScale;
+    return c;
+}
+
+// ---------------------------------------------------------------- phase B
+
+__device__ void phase_kstats_vencode(const QuantArgs& a, QuantShared& sh, uint64_t keep,
+                                     uint64_t release) {
+    if (threadIdx.x == 0) sh.qhead = 0u;
+    const float sV = tensor_scale_and_table(a.vpart, sh);     // (its barriers publish qhead)
+    if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scales[1] = sV;
+    const EncodeConsts c = encode_consts(sV);
+    // CTA b owns an even slice of the statistics units and of the V units;
+    // its warps take them from a shared-memory queue, statistics first
+    // (memory-bound) and V encoding after (arithmetic), so every SM
+    // interleaves K's HBM stream with V's arithmetic and no warp idles.
+    const int G = gridDim.x, b = blockIdx.x;
+    const int n_stats = a.nseg * a.ngroups;
+    const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
+    const int n_v = a.H * tiles;
+    const int s0 = (int)((long long)n_stats * b / G), s1 = (int)((long long)n_stats * (b + 1) / G);
+    const int v0 = (int)((long long)n_v * b / G), v1 = (int)((long long)n_v * (b + 1) / G);
+    const unsigned n_mine = (unsigned)((s1 - s0) + (v1 - v0));
+    const int lane = threadIdx.x & 31;
+    unsigned i = 0;
+    if (lane == 0) i = atomicAdd(&sh.qhead, 1u);
+    i = __shfl_sync(0xFFFFFFFFu, i, 0);
+    while (i < n_mine) {
+        unsigned next = 0;
+        if (lane == 0) next = atomicAdd(&sh.qhead, 1u);
+        if ((int)i < s1 - s0) {
+            stats_unit(a, s0 + (int)i, keep);
+        } else {
+            const int u = v0 + (int)i - (s1 - s0);
+            const int h = u / tiles;
+            const int tile = u - h * tiles;
+            encode_unit(a, sh, false, h, tile * kEncTokens, c.s, c.fast, c.ms6, c.ms4, c.rm,
+                               release);
+        }
+        i = __shfl_sync(0xFFFFFFFFu, next, 0);
+    }
+}
+
+// ---------------------------------------------------------------- phase C
+
+__device__ void phase_finalize(const QuantArgs& a, QuantShared& sh) {
+    float kp = 0.0f;
+    const int nblocks = a.HD / kFinCols;
+    const float Tf = (float)a.T;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const unsigned short* pmin = reinterpret_cast<const unsigned short*>(a.pmin);
+    const unsigned short* pmax = reinterpret_cast<const unsigned short*>(a.pmax);
+    for (int b = blockIdx.x; b < nblocks; b += gridDim.x) {
+        const int col = b * kFinCols + lane;
+        float S = 0.0f, mn = INFINITY, mx = -INFINITY;
+        for (int s0 = 0; s0 < a.nseg; s0 += kFinSegs) {
+            const int ns = min(kFinSegs, a.nseg - s0);
+            // all warps stage the pass's segments, every load in flight at once ...
+            float ps[kFinSegs / kQuantWarps];
+            unsigned short pn[kFinSegs / kQuantWarps], px[kFinSegs / kQuantWarps];
+#pragma unroll
+            for (int j = 0; j < kFinSegs / kQuantWarps; ++j) {
+                const int k = warp + j * kQuantWarps;
+                if (k < ns) {
+                    const size_t i = (size_t)(s0 + k) * a.HD + col;
+                    ps[j] = __ldcg(a.psum + i);
+                    pn[j] = __ldcg(pmin + i);
+                    px[j] = __ldcg(pmax + i);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kFinSegs / kQuantWarps; ++j) {
+                const int k = warp + j * kQuantWarps;
+                if (k < ns) {
+                    sh.fsum[k][lane] = ps[j];
+                    sh.fmin[k][lane] = pn[j];
+                    sh.fmax[k][lane] = px[j];
+                }
+            }
+            __syncthreads();
+            // ... and warp 0 adds them in segment order
+            if (warp == 0) {
+                for (int k = 0; k < ns; ++k) {
+                    S = __fadd_rn(S, sh.fsum[k][lane]);
+                    mn = fminf(mn, __uint_as_float((uint32_t)sh.fmin[k][lane] << 16));
+                    mx = fmaxf(mx, __uint_as_float((uint32_t)sh.fmax[k][lane] << 16));
+                }
+            }
+            __syncthreads();
+        }
+        if (warp == 0) {
+            const float mu = __fdiv_rn(S, Tf);
+            a.k_mean[col] = mu;
+            kp = fmaxf(kp, fmaxf(fabsf(__fsub_rn(mx, mu)), fabsf(__fsub_rn(mn, mu))));
+        }
+    }
+    const float b = block_max(kp, sh.red);
+    if (threadIdx.x == 0) a.kpart[blockIdx.x] = b;
+}
+
+// ---------------------------------------------------------------- phase D
+
+__device__ void phase_kencode(const QuantArgs& a, QuantShared& sh, uint64_t release) {
+    const float sK = tensor_scale_and_table(a.kpart, sh);
+    if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scales[0] = sK;
+    const EncodeConsts c = encode_consts(sK);
     const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     const int nw = gridDim.x * kQuantWarps;
-    const int tiles = (a.T + 15) / 16;
-    const int upt = a.H * tiles;
-    const int c8 = lane & 15;                 // 8-channel group of this lane
-    const bool odd = (lane & 1) != 0;         // second half of its 16-block
-    for (int u = wg; u < 2 * upt; u += nw) {
-        const bool isK = u < upt;
-        const int uu = isK ? u : u - upt;
-        const int h = uu / tiles;
-        const int tile = uu - h * tiles;
-        const float s = isK ? sK : sV;
-        // this lane's target: 6 on the even lane of a pair, 4 on the odd one
-        const float ms = __fmul_rn(odd ? 4.0f : 6.0f, s);
-        float mu[8];
-        if (isK) {
-            const float4* mp = reinterpret_cast<const float4*>(a.k_mean + h * kHeadDim + c8 * 8);
-            const float4 m0 = __ldcg(mp), m1 = __ldcg(mp + 1);
-            mu[0] = m0.x; mu[1] = m0.y; mu[2] = m0.z; mu[3] = m0.w;
-            mu[4] = m1.x; mu[5] = m1.y; mu[6] = m1.z; mu[7] = m1.w;
-        }
-        const uint4* src = isK ? a.K : a.V;
-        uint32_t* codes = reinterpret_cast<uint32_t*>(isK ? a.k_codes : a.v_codes);
-        uint8_t* scales = isK ? a.k_scales : a.v_scales;
-#pragma unroll 2
-        for (int it = 0; it < 8; ++it) {
-            const int t = tile * 16 + it * 2 + (lane >> 4);
-            const bool valid = t < a.T;
-            const uint4 w = valid ? ld_stream(src + ((size_t)t * a.H + h) * 16 + c8)
-                                  : make_uint4(0u, 0u, 0u, 0u);
-            float x[8];
-            unpack_bf16x8(w, x);
-            if (isK) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) x[i] = __fsub_rn(x[i], mu[i]);
-            }
-            float ah = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ah = fmaxf(ah, fabsf(x[i]));
-            const float ab = fmaxf(ah, __shfl_xor_sync(0xFFFFFFFFu, ah, 1));
-            // block scale for this lane's target, then swap with the partner
-            const float ratio = __fdiv_rn(ab, ms);
-            const uint32_t sb = cvt_e4m3x2(ratio, 0.0f) & 0xFFu;
-            const float D = __fmul_rn(e4m3_to_f32(sb), s);
-            const float r = D > 0.0f ? __frcp_rn(D) : 0.0f;
-            const float Do = __shfl_xor_sync(0xFFFFFFFFu, D, 1);
-            const float ro = __shfl_xor_sync(0xFFFFFFFFu, r, 1);
-            const uint32_t sbo = __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
-            const float D6 = odd ? Do : D, r6 = odd ? ro : r;
-            const float D4 = odd ? D : Do, r4 = odd ? r : ro;
-            const uint32_t sb6 = odd ? sbo : sb, sb4 = odd ? sb : sbo;
-            uint32_t q6, q4;
-            float e6, e4;
-            encode_half(x, D6, r6, q6, e6);
-            encode_half(x, D4, r4, q4, e4);
-            // block error = (elements 0..7) + (elements 8..15)
-            const float E6 = __fadd_rn(e6, __shfl_xor_sync(0xFFFFFFFFu, e6, 1));
-            const float E4 = __fadd_rn(e4, __shfl_xor_sync(0xFFFFFFFFu, e4, 1));
-            const bool keep4 = E4 < E6;
-            if (valid) {
-                const size_t row = (size_t)h * a.T + t;
-                codes[row * 16 + c8] = keep4 ? q4 : q6;
-                if (!odd) scales[row * 8 + (c8 >> 1)] = (uint8_t)(keep4 ? sb4 : sb6);
-            }
-        }
+    const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
+    for (int u = wg; u < a.H * tiles; u += nw) {
+        const int h = u / tiles;
+        const int tile = u - h * tiles;
+        encode_unit(a, sh, true, h, tile * kEncTokens, c.s, c.fast, c.ms6, c.ms4, c.rm, release);
     }
 }
 
-__global__ void __launch_bounds__(kQuantThreads, 2) quantize_kernel(QuantArgs a) {
-    __shared__ float red[kQuantWarps];
-    phase_stats(a, red);
+// CTA 0 records when it starts, when it finishes its share of each phase and
+// when it leaves each grid barrier (then the last CTA has arrived): a
+// per-phase profile of the launch.
+__device__ __forceinline__ void stamp(const QuantArgs& a, int i) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) a.ctl->stamp[i] = globaltimer_ns();
+}
+
+__global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a) {
+    __shared__ QuantShared sh;
+    const uint64_t keep = policy_keep(), release = policy_release();
+    stamp(a, 0);
+    phase_vmax(a, sh, keep);
+    stamp(a, 1);
     if (!grid_barrier(a.ctl)) return;
-    phase_finalize(a, red);
+    stamp(a, 2);
+    phase_kstats_vencode(a, sh, keep, release);
+    stamp(a, 3);
     if (!grid_barrier(a.ctl)) return;
-    phase_encode(a, red);
+    stamp(a, 4);
+    phase_finalize(a, sh);
+    stamp(a, 5);
+    if (!grid_barrier(a.ctl)) return;
+    stamp(a, 6);
+    phase_kencode(a, sh, release);
+    stamp(a, 7);
 }
 
 // ---------------------------------------------------------------- dequantize
@@ -433,6 +698,7 @@ nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
     a.kpart = reinterpret_cast<float*>(w + L.kpart);
     a.vpart = reinterpret_cast<float*>(w + L.vpart);
     a.ctl = reinterpret_cast<Control*>(w);
+    a.one = 1.0f;
     void* args[] = {&a};
     cudaError_t e = cudaLaunchCooperativeKernel((const void*)quantize_kernel,
                                                 dim3(g_quant_grid[dev]), dim3(kQuantThreads),

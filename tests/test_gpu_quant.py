@@ -68,6 +68,43 @@ def test_degenerate_inputs_bit_exact(lib, orc):
         _assert_same(out.to_host(), orc.quantize_chunk(K, V), what)
 
 
+def _bf16_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_signed_zeros_subnormals_and_extreme_magnitudes_bit_exact(lib, orc):
+    """Cases the fast division path must reproduce exactly: -0 inside blocks
+    with a nonzero scale (the code keeps the sign), bf16 subnormals, whole
+    tensors scaled to 2^-110 and 2^100, and single blocks scaled to 2^-110
+    inside an ordinary tensor (their block max is below the fast-path bound)."""
+    T, H = 200, 3
+    rng = np.random.default_rng(11)
+    K = synth.k_with_offsets_bf16(61, T, H, (T, H, 128))
+    V = synth.gaussian_bf16(61, T, H, synth.T_V, (T, H, 128))
+    cases = []
+    # exact -0 in V, and a K channel of signed zeros: its mean is +0, so
+    # RN(-0 - mean) = -0 reaches the encoder
+    Vz = V.copy()
+    Vz[rng.random(V.shape) < 0.05] = 0x8000
+    Kz = K.copy()
+    Kz[:, :, 5] = np.where(rng.random((T, H)) < 0.5, 0x8000, 0x0000).astype(np.uint16)
+    cases.append((Kz, Vz, "signed zeros"))
+    Vs = V.copy()
+    m = rng.random(V.shape) < 0.03
+    Vs[m] = (rng.integers(1, 0x80, m.sum()) | (rng.integers(0, 2, m.sum()) << 15)).astype(np.uint16)
+    cases.append((K, Vs, "bf16 subnormals"))
+    for e in (-110, 100):
+        cases.append((synth.to_bf16_bits(_bf16_to_f64(K) * 2.0 ** e),
+                      synth.to_bf16_bits(_bf16_to_f64(V) * 2.0 ** e), f"scaled by 2^{e}"))
+    blocks = rng.random((T, H, 8)) < 0.02
+    scale = np.where(np.repeat(blocks, 16, axis=2), 2.0 ** -110, 1.0)
+    cases.append((synth.to_bf16_bits(_bf16_to_f64(K) * scale),
+                  synth.to_bf16_bits(_bf16_to_f64(V) * scale), "tiny blocks"))
+    for K_, V_, what in cases:
+        out, _ = _gpu_quant(lib, K_, V_)
+        _assert_same(out.to_host(), orc.quantize_chunk(K_, V_), what)
+
+
 def test_repeated_calls_share_one_workspace(lib, orc):
     ws = None
     for i in range(3):
