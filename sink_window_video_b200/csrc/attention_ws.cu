@@ -11,25 +11,31 @@
 // into fp16 range.
 //
 // One CTA per SM: a head and 256 query rows (two 128-row tiles Q0, Q1), keys
-// in 64-key tiles.  Warp roles (352 threads; 11 warps keep 168 registers per
+// in 128-key tiles.  Warp roles (352 threads; 11 warps keep 168 registers per
 // thread, registers being split among the four SM sub-partitions):
 //   warps 0-3   softmax of Q0 (thread = row = TMEM lane)
 //   warps 4-7   softmax of Q1
 //   warp 8      tensor memory allocation and the MMA issue (one thread)
-//   warps 9-10  de-quantize K and V tiles (thread = key row) into a 4-stage
-//               shared-memory ring (128-byte-swizzled: K-major B of
+//   warps 9-10  de-quantize K and V tiles (two key rows per thread) into a
+//               2-stage shared-memory ring (128-byte-swizzled: K-major B of
 //               S = Q K^T, MN-major B of P V)
-// (warp w runs on SM sub-partition w mod 4: each carries two softmax warps,
-// and the issue and conversion work of the other roles is spread over three.)
-// Tensor memory (512 columns): Q0 | Q1 (fp16, 64 each; the A operand of
-// S = Q K^T) | S0 | S1 (fp32, 64 each; P in fp16 over their first 32) |
-// O0 | O1 (fp32, 128 each).  With Q in tensor memory the MMAs read only B
-// from shared memory, which leaves shared-memory bandwidth for the
-// de-quantization stores.
+// (warp w runs on SM sub-partition w mod 4.)
+// Tile size: every tcgen05.mma of M = 128, K = 16 costs about the same issue
+// time up to N = 128, so the products run at N = 128 -- 128 keys for Q K^T and
+// d = 128 for P V -- halving the instruction count of 64-key tiles.
+// Shared memory (192 KB): Q0, Q1 (fp16, the A operand of S = Q K^T, K-major)
+// and the ring of K / V tiles.
+// Tensor memory (512 columns): S0 | S1 (fp32, 128 each; P in fp16 over their
+// first 64) | O0 | O1 (fp32, 128 each).
 // MMA order per key tile t:  PV0(t) QK0(t+1) | PV1(t) QK1(t+1); while one
 // softmax group works on S_i, the tensor core runs the other group's
 // products.  P_i over S_i is safe because tcgen05 MMAs of one thread execute
 // in issue order.
+// Softmax per tile, per row, in two 64-key halves: the half's max decides
+// lazily whether the reference max moves (only when it grows by more than
+// 2^8; then O, the row sum and the tile's first P half are rescaled); six of
+// every eight exponential pairs on the special-function unit, two on the FMA
+// pipe.
 // Synchronization is by mbarriers only: kv_full/kv_empty (ring), s_full
 // (S_i ready; its commit also covers the previous PV_i, so O_i is quiescent
 // for a rescale), p_full (P_i written), q_ready, o_final.  Every wait is
@@ -45,14 +51,14 @@ namespace nvfp4kv {
 using namespace tc;
 namespace {
 
-constexpr int kKeysW = 64;                  // keys per tile
-constexpr int kStages = 4;                  // de-quantized K/V ring depth
+constexpr int kKeysW = 128;                 // keys per tile
+constexpr int kStages = 2;                  // de-quantized K/V ring depth
 constexpr int kThreadsW = 352;
 constexpr int kMmaWarp = 8;
 constexpr int kDequantWarp0 = 9;
-constexpr uint32_t kColQ = 0, kColS = 128, kColO = 256, kColsW = 512;
-constexpr int kStageBytes = kKeysW * 128 * 2;            // 16 KB per operand tile
-constexpr size_t kSmemW = 2 * kStages * kStageBytes + 1024;
+constexpr uint32_t kColS = 0, kColO = 256, kColsW = 512;
+constexpr int kTileB = 128 * 128 * 2;                    // 32 KB fp16 operand tile
+constexpr size_t kSmemW = (2 + 2 * kStages) * kTileB + 1024;
 constexpr float kLog2eW = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -108,34 +114,30 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t mbar, uint32_t parity, vo
     }
 }
 
-// K-major, 64-key, 128-byte-swizzled operand: key row kl, 16-byte chunk c of
-// d (0..15).  Two 8 KB blocks along d.
-__device__ __forceinline__ uint32_t kv_off(int kl, int c) {
-    return (uint32_t)((c >> 3) * 8192 + kl * 128 + (((c & 7) ^ (kl & 7)) << 4));
-}
-
-// De-quantize 64 consecutive codes (32 bytes) with their 4 block scales into
-// chunks 8*half .. 8*half+7 of key row kl of a swizzled tile.
-__device__ __forceinline__ void dequant_half(const uint4 c0, const uint4 c1, uint32_t sc,
-                                             uint8_t* tile, int kl, int half) {
-    const uint32_t s01 = cvt_e4m3x2_to_f16x2(sc & 0xFFFFu);
-    const uint32_t s23 = cvt_e4m3x2_to_f16x2(sc >> 16);
-    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+// De-quantize one 128-channel row (64 code bytes, 8 E4M3 scale bytes, held in
+// registers) to fp16 into row r of a swizzled [2][128][128 B] tile.
+__device__ __forceinline__ void dequant_row_regs(const uint4* cw4, uint2 sc, uint8_t* tile, int r) {
+    const uint32_t s01 = cvt_e4m3x2_to_f16x2(sc.x & 0xFFFFu);
+    const uint32_t s23 = cvt_e4m3x2_to_f16x2(sc.x >> 16);
+    const uint32_t s45 = cvt_e4m3x2_to_f16x2(sc.y & 0xFFFFu);
+    const uint32_t s67 = cvt_e4m3x2_to_f16x2(sc.y >> 16);
+    const uint32_t sp[4] = {s01, s23, s45, s67};
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {            // block b: code words 2b, 2b+1
-        const uint32_t pair = (b < 2) ? s01 : s23;
-        const uint32_t sh = (b & 1) ? (pair >> 16) : (pair & 0xFFFFu);
-        const uint32_t s2 = sh | (sh << 16);
+    for (int b = 0; b < 8; ++b) {            // block b: code words 2b, 2b+1 -> chunks 2b, 2b+1
+        const uint32_t pair = sp[b >> 1];
+        const uint32_t shv = (b & 1) ? (pair >> 16) : (pair & 0xFFFFu);
+        const uint32_t s2 = shv | (shv << 16);
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-            uint32_t h[4];
-            cvt_e2m1x8_to_f16x2(cw[2 * b + w], h);
+            const uint32_t word = (&cw4[b >> 1].x)[(b & 1) * 2 + w];
+            uint32_t hh[4];
+            cvt_e2m1x8_to_f16x2(word, hh);
             uint4 o;
-            o.x = hmul2_u32(h[0], s2);
-            o.y = hmul2_u32(h[1], s2);
-            o.z = hmul2_u32(h[2], s2);
-            o.w = hmul2_u32(h[3], s2);
-            *reinterpret_cast<uint4*>(tile + kv_off(kl, half * 8 + 2 * b + w)) = o;
+            o.x = hmul2_u32(hh[0], s2);
+            o.y = hmul2_u32(hh[1], s2);
+            o.z = hmul2_u32(hh[2], s2);
+            o.w = hmul2_u32(hh[3], s2);
+            *reinterpret_cast<uint4*>(tile + sw128_off(r, 2 * b + w)) = o;
         }
     }
 }
@@ -184,8 +186,9 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
 
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t* Kt = base;                                  // [kStages][16 KB]
-    uint8_t* Vt = base + kStages * kStageBytes;          // [kStages][16 KB]
+    uint8_t* Qt = base;                                   // [2][32 KB]
+    uint8_t* Kt = base + 2 * kTileB;                      // [kStages][32 KB]
+    uint8_t* Vt = Kt + kStages * kTileB;                  // [kStages][32 KB]
 
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -218,14 +221,13 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         const int qi = warp >> 2;                          // query tile 0 or 1
         const int r = tid & 127;                           // row in the tile
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tQ = tmem + lane_base + kColQ + 64u * qi;
-        const uint32_t tS = tmem + lane_base + kColS + 64u * qi;
+        const uint32_t tS = tmem + lane_base + kColS + 128u * qi;
         const uint32_t tO = tmem + lane_base + kColO + 128u * qi;
         const int row = m0 + qi * 128 + r;
         const bool rvalid = row < a.T_q;
         const uint4* qsrc = reinterpret_cast<const uint4*>(a.Q + ((size_t)row * H + h) * kHeadDim);
 
-        // Q row -> fp16 (scaled by 2^-e into range) -> tensor memory (A of Q K^T)
+        // Q row -> fp16 (scaled by 2^-e into range), swizzled K-major into smem
         float qexp;
         {
             uint4 w[16];
@@ -245,19 +247,20 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
             if (amax_bits != 0) e = max(-120, min(120, (int)(amax_bits >> 23) - 127 - 14));
             const float down = __uint_as_float((uint32_t)(127 - e) << 23);
             qexp = __uint_as_float((uint32_t)(127 + e) << 23);
-            uint32_t qh[64];
+            uint8_t* qt = Qt + qi * kTileB;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 float f[8];
                 unpack_bf16x8(w[c], f);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) qh[4 * c + j] = pack_f16x2(f[2 * j] * down, f[2 * j + 1] * down);
+                uint4 o;
+                o.x = pack_f16x2(f[0] * down, f[1] * down);
+                o.y = pack_f16x2(f[2] * down, f[3] * down);
+                o.z = pack_f16x2(f[4] * down, f[5] * down);
+                o.w = pack_f16x2(f[6] * down, f[7] * down);
+                *reinterpret_cast<uint4*>(qt + sw128_off(r, c)) = o;
             }
-            tmem_st32(tQ, qh);
-            tmem_st32(tQ + 32, qh + 32);
-            tmem_wait_st();
         }
-        tc_fence_before();
+        fence_async_smem();
         mbar_arrive(smem_u32(&sh.q_ready[qi]));
 
         float sVmax = 0.0f;
@@ -295,72 +298,101 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                 bool got = wait_or_abort(s_full, (uint32_t)(t & 1), abort, a.ctl, 10u + qi, t);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t s[64];
-                __syncwarp();
-                tmem_ld32(tS, s);
-                tmem_ld32(tS + 32, s + 32);
-                tmem_wait_ld();
                 const int valid = min(kKeysW, T_c - j0);
-                if (valid < kKeysW) {
-#pragma unroll
-                    for (int k = 0; k < 64; ++k)
-                        if (k >= valid) s[k] = __float_as_uint(-INFINITY);
-                }
-                // row max: eight independent chains, then a short tree
-                float m8[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) m8[c] = fmaxf(__uint_as_float(s[c]), __uint_as_float(s[c + 8]));
-#pragma unroll
-                for (int k = 16; k < 64; k += 16)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        m8[c] = fmax3(m8[c], __uint_as_float(s[k + c]), __uint_as_float(s[k + 8 + c]));
-                float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
-                                 fmaxf(m8[6], m8[7]));
-                mx = fmaf(mx, alpha, beta);                 // alpha > 0: same argmax
-                const bool grow = mx > m_run + kRescaleLog2 || m_run == -INFINITY;
-                float corr = 1.0f;
-                if (grow) {
-                    const float m_new = fmaxf(mx, m_run);
-                    corr = ex2f(m_run - m_new);
-                    l_run *= corr;
-                    m_run = m_new;
-                }
-                if (o_written && __any_sync(0xFFFFFFFFu, grow)) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t ov[32];
-                        tmem_ld32(tO + 32 * q, ov);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-                        tmem_st32(tO + 32 * q, ov);
-                    }
-                }
-                // p' = 2^(logit - m + log2(s_V/s_Vmax)), one fused multiply-add each
-                // two of every eight pairs on the FMA pipe, the rest on the
-                // special-function unit; four independent partial sums
-                const float b2 = beta - m_run + lrV;
-                const float2 b22 = make_float2(b2, b2);
                 float2 acc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                                  make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-                uint32_t p[32];
+                // two 64-key halves; P of half hh (fp16) goes to columns
+                // 32 hh .. 32 hh + 31, over S columns already read
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t s[64];
+                    __syncwarp();
+                    tmem_ld32(tS + 64 * hh, s);
+                    tmem_ld32(tS + 64 * hh + 32, s + 32);
+                    tmem_wait_ld();
+                    const int vh = valid - 64 * hh;            // valid keys of this half
+                    if (vh < 64) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    float2 z = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])),
-                                          alpha2, b22);
-                    if ((k & 7) >= 6) {
-                        z = ex2_poly2(z);
-                    } else {
-                        z.x = ex2f(z.x);
-                        z.y = ex2f(z.y);
+                        for (int k = 0; k < 64; ++k)
+                            if (k >= vh) s[k] = __float_as_uint(-INFINITY);
                     }
-                    acc[k & 3] = __fadd2_rn(acc[k & 3], z);
-                    p[k] = pack_f16x2(z.x, z.y);
+                    // row max: eight independent chains, then a short tree
+                    float m8[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) m8[c] = fmaxf(__uint_as_float(s[c]), __uint_as_float(s[c + 8]));
+#pragma unroll
+                    for (int k = 16; k < 64; k += 16)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            m8[c] = fmax3(m8[c], __uint_as_float(s[k + c]), __uint_as_float(s[k + 8 + c]));
+                    float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                                     fmaxf(m8[6], m8[7]));
+                    mx = fmaf(mx, alpha, beta);                 // alpha > 0: same argmax
+                    // (a half without valid keys has mx = -inf and never grows)
+                    const bool grow = mx > m_run + kRescaleLog2 || (m_run == -INFINITY && mx > -INFINITY);
+                    float corr = 1.0f;
+                    if (grow) {
+                        const float m_new = fmaxf(mx, m_run);
+                        corr = ex2f(m_run - m_new);
+                        l_run *= corr;
+                        m_run = m_new;
+                    }
+                    if (__any_sync(0xFFFFFFFFu, grow)) {
+                        // rare: rescale what this row holds with the old max --
+                        // O (if written), this tile's first P half and sums
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            acc[i].x *= corr;
+                            acc[i].y *= corr;
+                        }
+                        if (o_written) {
+#pragma unroll 1
+                            for (int q = 0; q < 4; ++q) {
+                                uint32_t ov[32];
+                                tmem_ld32(tO + 32 * q, ov);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+                                tmem_st32(tO + 32 * q, ov);
+                            }
+                        }
+                        if (hh == 1) {
+                            tmem_wait_st();                     // the first half's P is written
+                            const uint32_t c2 = pack_f16x2(corr, corr);
+#pragma unroll 1
+                            for (int q = 0; q < 2; ++q) {
+                                uint32_t pv[16];
+                                tmem_ld16(tS + 16 * q, pv);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) pv[i] = hmul2_u32(pv[i], c2);
+                                tmem_st16(tS + 16 * q, pv);
+                            }
+                        }
+                    }
+                    // p' = 2^(logit - m + log2(s_V/s_Vmax)), one fused multiply-add each;
+                    // two of every eight pairs on the FMA pipe, the rest on the
+                    // special-function unit; four independent partial sums
+                    const float b2 = beta - m_run + lrV;
+                    const float2 b22 = make_float2(b2, b2);
+                    uint32_t p[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        float2 z = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])),
+                                              alpha2, b22);
+                        if ((k & 7) >= 6) {
+                            z = ex2_poly2(z);
+                        } else {
+                            z.x = ex2f(z.x);
+                            z.y = ex2f(z.y);
+                        }
+                        acc[k & 3] = __fadd2_rn(acc[k & 3], z);
+                        p[k] = pack_f16x2(z.x, z.y);
+                    }
+                    __syncwarp();
+                    tmem_st32(tS + 32 * hh, p);
                 }
-                __syncwarp();
-                tmem_st32(tS, p);
                 tmem_wait_st();
                 const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
                 const float2 a03 = __fadd2_rn(a01, a23);
@@ -410,83 +442,84 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         }
     } else if (warp >= kDequantWarp0) {
         // ------------------------------------------------------------ de-quantize
-        // One thread per key row; the codes and scales of tile t+1 are loaded
-        // into registers before tile t is converted, so the L2 latency of the
-        // loads overlaps one tile period.
-        const int kl = tid - kDequantWarp0 * 32;           // key row 0..63
+        // Each thread converts key rows kl and kl + 64.  A row's codes and
+        // scales for the next tile are loaded right after the row is
+        // converted, so the L2 latency overlaps the rest of the tile period.
+        // Rows past a chunk's end get zero codes and zero scales: exact zeros.
+        const int kl = tid - kDequantWarp0 * 32;           // 0..63
         struct Packed {
             uint4 kc[4], vc[4];
             uint2 ks, vs;
         };
-        auto load_tile = [&](int t, Packed& p) {
-            const int ci = t / tiles_per_chunk;
-            const int key = (t - ci * tiles_per_chunk) * kKeysW + kl;
-            if (t < ntiles && key < T_c) {
+        auto load_row = [&](int tt, int row, Packed& pk) {
+            const int ci = tt / tiles_per_chunk;
+            const int key = (tt - ci * tiles_per_chunk) * kKeysW + row;
+            if (tt < ntiles && key < T_c) {
                 const WsChunk& cp = a.chunk[ci];
                 const size_t rowi = (size_t)h * T_c + key;
                 const uint4* kp = reinterpret_cast<const uint4*>(cp.k_codes + rowi * 64);
                 const uint4* vp = reinterpret_cast<const uint4*>(cp.v_codes + rowi * 64);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) { p.kc[i] = kp[i]; p.vc[i] = vp[i]; }
-                p.ks = *reinterpret_cast<const uint2*>(cp.k_scales + rowi * 8);
-                p.vs = *reinterpret_cast<const uint2*>(cp.v_scales + rowi * 8);
+                for (int i = 0; i < 4; ++i) { pk.kc[i] = kp[i]; pk.vc[i] = vp[i]; }
+                pk.ks = *reinterpret_cast<const uint2*>(cp.k_scales + rowi * 8);
+                pk.vs = *reinterpret_cast<const uint2*>(cp.v_scales + rowi * 8);
             } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) p.kc[i] = p.vc[i] = make_uint4(0, 0, 0, 0);
-                p.ks = p.vs = make_uint2(0, 0);
+                for (int i = 0; i < 4; ++i) pk.kc[i] = pk.vc[i] = make_uint4(0, 0, 0, 0);
+                pk.ks = pk.vs = make_uint2(0, 0);
             }
         };
-        Packed cur, nxt;
-        load_tile(0, cur);
+        Packed ra, rb;
+        load_row(0, kl, ra);
+        load_row(0, kl + 64, rb);
         for (int t = 0; t < ntiles; ++t) {
             const int st = t % kStages;
-            load_tile(t + 1, nxt);
             if (t >= kStages) {
                 bool got = wait_or_abort(smem_u32(&sh.kv_empty[st]),
                                          (uint32_t)(((t / kStages) - 1) & 1), abort, a.ctl, 30u, t);
                 if (!__all_sync(0xFFFFFFFFu, got)) break;
             }
-            uint8_t* kt = Kt + st * kStageBytes;
-            uint8_t* vt = Vt + st * kStageBytes;
-            // rows past the chunk's end are zero codes and zero scales: exact zeros
-            dequant_half(cur.kc[0], cur.kc[1], cur.ks.x, kt, kl, 0);
-            dequant_half(cur.kc[2], cur.kc[3], cur.ks.y, kt, kl, 1);
-            dequant_half(cur.vc[0], cur.vc[1], cur.vs.x, vt, kl, 0);
-            dequant_half(cur.vc[2], cur.vc[3], cur.vs.y, vt, kl, 1);
+            uint8_t* kt = Kt + st * kTileB;
+            uint8_t* vt = Vt + st * kTileB;
+            dequant_row_regs(ra.kc, ra.ks, kt, kl);
+            dequant_row_regs(ra.vc, ra.vs, vt, kl);
+            load_row(t + 1, kl, ra);
+            dequant_row_regs(rb.kc, rb.ks, kt, kl + 64);
+            dequant_row_regs(rb.vc, rb.vs, vt, kl + 64);
+            load_row(t + 1, kl + 64, rb);
             fence_async_smem();
             mbar_arrive(smem_u32(&sh.kv_full[st]));
-            cur = nxt;
         }
     } else if (lane == 0) {
         // ------------------------------------------------------------ MMA issue (warp 8)
-        constexpr uint32_t idesc_qk = umma_idesc_f16(false, 64);
+        constexpr uint32_t idesc_qk = umma_idesc_f16(false, 128);
         constexpr uint32_t idesc_pv = umma_idesc_f16(true, 128);
-        const uint32_t kt_addr = smem_u32(Kt), vt_addr = smem_u32(Vt);
+        // Descriptors of the first tiles; a tile or k-step offset is added to
+        // the start-address field (bits 0..13, address >> 4): shared-memory
+        // addresses stay below 256 KB, so the field never carries.
+        const uint64_t qdesc0 = umma_desc(smem_u32(Qt), 16, 1024);
+        const uint64_t kdesc0 = umma_desc(smem_u32(Kt), 16, 1024);
+        const uint64_t vdesc0 = umma_desc(smem_u32(Vt), 16384, 1024);
         bool ok = wait_or_abort(smem_u32(&sh.q_ready[0]), 0u, abort, a.ctl, 40u, 0) &&
                   wait_or_abort(smem_u32(&sh.q_ready[1]), 0u, abort, a.ctl, 41u, 0);
-        // Descriptors of stage 0; a stage or k-step offset is added to the
-        // start-address field (bits 0..13, address >> 4): shared-memory
-        // addresses stay below 256 KB, so the field never carries.
-        const uint64_t kdesc0 = umma_desc(kt_addr, 16, 1024);
-        const uint64_t vdesc0 = umma_desc(vt_addr, 8192, 1024);
         auto issue_qk = [&](int qi, int st) {
-            const uint64_t d0 = kdesc0 + (uint64_t)((st * kStageBytes) >> 4);
-            const uint32_t dt = tmem + kColS + 64u * qi;
-            const uint32_t at = tmem + kColQ + 64u * qi;
+            const uint64_t qd = qdesc0 + (uint64_t)((qi * kTileB) >> 4);
+            const uint64_t kd = kdesc0 + (uint64_t)((st * kTileB) >> 4);
+            const uint32_t dt = tmem + kColS + 128u * qi;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_ts(dt, at + (uint32_t)(ks * 8),
-                       d0 + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), idesc_qk,
-                       ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                mma_ss(dt, qd + off, kd + off, idesc_qk, ks > 0 ? 1u : 0u);
+            }
             mma_commit(smem_u32(&sh.s_full[qi]));
         };
         auto issue_pv = [&](int qi, int st, bool first) {
-            const uint64_t d0 = vdesc0 + (uint64_t)((st * kStageBytes) >> 4);
+            const uint64_t vd = vdesc0 + (uint64_t)((st * kTileB) >> 4);
             const uint32_t dt = tmem + kColO + 128u * qi;
-            const uint32_t at = tmem + kColS + 64u * qi;
+            const uint32_t at = tmem + kColS + 128u * qi;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_ts(dt, at + (uint32_t)(ks * 8), d0 + (uint64_t)((ks * 2048) >> 4), idesc_pv,
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ts(dt, at + (uint32_t)(ks * 8), vd + (uint64_t)((ks * 2048) >> 4), idesc_pv,
                        (ks > 0 || !first) ? 1u : 0u);
         };
         if (ok) {
