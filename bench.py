@@ -311,7 +311,8 @@ def run_ours(args, rank, world, local):
         rollouts = [run_rollout(swv, cfg, pool, O, stream, world) for cfg in ROLLOUTS]
 
     return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
-                e2e_ms=e2e_ms, rollouts=rollouts)
+                e2e_ms=e2e_ms, rollouts=rollouts,
+                attn_launches=swv.attention_launches(len(cache.keyset(0)), T, H, T))
 
 
 # ------------------------------------------------------------------ rollouts
@@ -369,7 +370,7 @@ def run_rollout(swv, cfg, pool, O, stream, world):
                          f"S_g={cfg['S_g']}, S_s={cfg['S_s']}, W={cfg['W']}, shot switches at "
                          f"{list(cfg['switches']) or 'none'}"),
             "chunks_per_s": value, "ms": ms, "attention_flops": flops,
-            "gpu_launches": 2 * n_quant,
+            "gpu_launches": n_quant + sum(swv.attention_launches(k, T, H, T) for k in sizes) * layers,
             "quantizations": n_quant, "keyset_sizes": sizes,
             "roofline_chunks_per_s": chunks * world / t_roof, "frac": value * t_roof / (chunks * world),
             "roofline_basis": f"{src} bf16 sustained + {src} hbm, attention and quantizer serial"}
@@ -513,7 +514,7 @@ def main():
                          "ms_per_launch": r["ms_quant"], "peak_source": f"{peak_src} hbm"},
             "attention": {"ms_per_launch": r["ms_attn"], "flops_per_launch": attn_flops(),
                           "tflops": attn_tf},
-            "gpu_launches": 2 * K,
+            "gpu_launches": K * (1 + r["attn_launches"]),
             "clocks": r["clocks"],
         }
         if r["e2e_ms"] is not None:

@@ -100,8 +100,11 @@ nvfp4kv_status nvfp4kv_chunk_view_init(void* base, int T_c, int H, int d,
                                        nvfp4kv_chunk_view* out);
 
 /* Bytes of the scratch workspace the quantizer and the attention need for
- * chunks of this shape (partial sums of the K-smoothing mean, per-block
- * maxima, the grid barrier and the status word). */
+ * chunks of this shape: partial sums of the K-smoothing mean, per-block
+ * maxima, the grid barrier and the status word, and room for the attention's
+ * partial results when it splits the key range of its last query blocks
+ * (sized for up to T_c query rows; with more rows the attention runs
+ * unsplit). */
 size_t nvfp4kv_workspace_bytes(int T_c, int H, int d);
 
 /* Zero the workspace's control words (status, barrier) on `stream`.  Call it
@@ -195,6 +198,15 @@ nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
                                  int T_c, int H, int d, const void* Q, int T_q,
                                  void* O, int o_dtype, float softmax_scale, void* ws,
                                  nvfp4kv_stream_t stream);
+
+/*
+ * Number of kernels one attention call of this shape enqueues: 1, or 2 when
+ * the query blocks left over for the GPU's last, partial wave are split
+ * along the keys and merged by a second kernel (the split is an execution
+ * detail: the result is the same softmax attention).  0 for invalid sizes.
+ * Host-only; queries the current device's multiprocessor count once.
+ */
+int nvfp4kv_attention_launches(int n_chunks, int T_c, int H, int d, int T_q);
 
 /* ------------------------------------------------------------------ cache */
 

@@ -68,6 +68,7 @@ def load():
         "nvfp4kv_quantize_chunk": (st, [vp, vp, i32, i32, i32, cv, vp, vp]),
         "nvfp4kv_dequantize": (st, [cv, i32, i32, i32, vp, vp, i32, vp]),
         "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp]),
+        "nvfp4kv_attention_launches": (i32, [i32, i32, i32, i32, i32]),
         "kvcache_pool_bytes": (sz, [cfgp]),
         "kvcache_create": (st, [cfgp, vp, vp, ctypes.POINTER(vp)]),
         "kvcache_destroy": (None, [vp]),
@@ -130,6 +131,11 @@ def version() -> str:
 
 def chunk_bytes(T_c, H, d=HEAD_DIM) -> int:
     return int(load().nvfp4kv_chunk_bytes(T_c, H, d))
+
+
+def attention_launches(n_chunks, T_c, H, T_q, d=HEAD_DIM) -> int:
+    """Kernels one attention call of this shape enqueues (1, or 2 with a split tail)."""
+    return int(load().nvfp4kv_attention_launches(n_chunks, T_c, H, d, T_q))
 
 
 def workspace_bytes(T_c, H, d=HEAD_DIM) -> int:

@@ -161,6 +161,16 @@ nvfp4kv_status nvfp4kv_chunk_view_init(void* base, int T_c, int H, int d,
     return NVFP4KV_OK;
 }
 
+int nvfp4kv_attention_launches(int n_chunks, int T_c, int H, int d, int T_q) {
+    if (!valid_shape(T_c, H, d) || n_chunks < 1 || n_chunks > NVFP4KV_MAX_KEY_CHUNKS ||
+        T_q <= 0)
+        return 0;
+    const char* e = std::getenv("NVFP4KV_ATTENTION_KERNEL");
+    if (e != nullptr && (std::strcmp(e, "mma") == 0 || std::strcmp(e, "tc1") == 0)) return 1;
+    const AttnPlan p = attention_plan(n_chunks, T_c, H, T_q, ws_layout(T_c, H).apart_pairs);
+    return p.n_tail > 0 ? 2 : 1;
+}
+
 size_t nvfp4kv_workspace_bytes(int T_c, int H, int d) {
     if (!valid_shape(T_c, H, d)) return 0;
     return ws_layout(T_c, H).total;

@@ -79,6 +79,10 @@ struct WsArgs {
     int o_f32;
     float scale_log2;
     Control* ctl;
+    // work split: CTA b < n_full takes query block b whole; later CTAs take
+    // key range (b - n_full) % n_split of query block n_full + (b - n_full) / n_split
+    int pairs_per_head, n_full, n_split;
+    float* part;            // partial results of split blocks
 };
 
 struct WsShared {
@@ -177,11 +181,20 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int h = blockIdx.y;
-    const int m0 = blockIdx.x * 256;
+    const int item = blockIdx.x;
+    const bool split = item >= a.n_full;
+    const int piece = split ? item - a.n_full : 0;
+    const int pair = split ? a.n_full + piece / a.n_split : item;
+    const int q_split = split ? piece % a.n_split : 0;
+    const int n_ranges = split ? a.n_split : 1;
+    const int h = pair / a.pairs_per_head;
+    const int m0 = (pair - h * a.pairs_per_head) * 256;
     const int H = a.H, T_c = a.T_c;
     const int tiles_per_chunk = (T_c + kKeysW - 1) / kKeysW;
-    const int ntiles = a.n_chunks * tiles_per_chunk;
+    const int ntiles_all = a.n_chunks * tiles_per_chunk;
+    // this CTA's key tiles: global tile indices [t_begin, t_begin + ntiles)
+    const int t_begin = (int)((long long)ntiles_all * q_split / n_ranges);
+    const int ntiles = (int)((long long)ntiles_all * (q_split + 1) / n_ranges) - t_begin;
     volatile int* abort = &sh.abort;
 
     const uint32_t raw = smem_u32(smem_raw);
@@ -271,30 +284,38 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         int t = 0;
         const uint32_t s_full = smem_u32(&sh.s_full[qi]);
         const uint32_t p_full = smem_u32(&sh.p_full[qi]);
-        for (int ci = 0; ci < a.n_chunks && ok; ++ci) {
-            const WsChunk cp = a.chunk[ci];
-            const float sK = cp.tensor_scales[0], sV = cp.tensor_scales[1];
-            float qmu = 0.0f;
-            if (rvalid) {
-                const float4* mp = reinterpret_cast<const float4*>(cp.k_mean + h * kHeadDim);
+        int ci_cur = -1;
+        float alpha = 0.0f, beta = 0.0f, lrV = 0.0f, inv_rV = 0.0f;
+        float2 alpha2 = make_float2(0.0f, 0.0f);
+        for (; t < ntiles && ok; ++t) {
+            const int gt = t_begin + t;                        // global tile index
+            const int ci = gt / tiles_per_chunk;
+            const int j0 = (gt - ci * tiles_per_chunk) * kKeysW;
+            if (ci != ci_cur) {
+                ci_cur = ci;
+                const WsChunk cp = a.chunk[ci];
+                const float sK = cp.tensor_scales[0], sV = cp.tensor_scales[1];
+                float qmu = 0.0f;
+                if (rvalid) {
+                    const float4* mp = reinterpret_cast<const float4*>(cp.k_mean + h * kHeadDim);
 #pragma unroll 4
-                for (int c = 0; c < 16; ++c) {
-                    float f[8];
-                    unpack_bf16x8(qsrc[c], f);
-                    const float4 u0 = mp[2 * c], u1 = mp[2 * c + 1];
-                    qmu = fmaf(f[0], u0.x, qmu); qmu = fmaf(f[1], u0.y, qmu);
-                    qmu = fmaf(f[2], u0.z, qmu); qmu = fmaf(f[3], u0.w, qmu);
-                    qmu = fmaf(f[4], u1.x, qmu); qmu = fmaf(f[5], u1.y, qmu);
-                    qmu = fmaf(f[6], u1.z, qmu); qmu = fmaf(f[7], u1.w, qmu);
+                    for (int c = 0; c < 16; ++c) {
+                        float f[8];
+                        unpack_bf16x8(qsrc[c], f);
+                        const float4 u0 = mp[2 * c], u1 = mp[2 * c + 1];
+                        qmu = fmaf(f[0], u0.x, qmu); qmu = fmaf(f[1], u0.y, qmu);
+                        qmu = fmaf(f[2], u0.z, qmu); qmu = fmaf(f[3], u0.w, qmu);
+                        qmu = fmaf(f[4], u1.x, qmu); qmu = fmaf(f[5], u1.y, qmu);
+                        qmu = fmaf(f[6], u1.z, qmu); qmu = fmaf(f[7], u1.w, qmu);
+                    }
                 }
+                alpha = qexp * sK * a.scale_log2;
+                beta = qmu * a.scale_log2;
+                lrV = __log2f(sV / sVmax);
+                inv_rV = sVmax / sV;
+                alpha2 = make_float2(alpha, alpha);
             }
-            const float alpha = qexp * sK * a.scale_log2;
-            const float beta = qmu * a.scale_log2;
-            const float lrV = __log2f(sV / sVmax);
-            const float inv_rV = sVmax / sV;
-            const float2 alpha2 = make_float2(alpha, alpha);
-
-            for (int j0 = 0; j0 < T_c; j0 += kKeysW, ++t) {
+            {
                 bool got = wait_or_abort(s_full, (uint32_t)(t & 1), abort, a.ctl, 10u + qi, t);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 tc_fence_after();
@@ -409,13 +430,23 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         if (ok) {
             tc_fence_after();
             const float inv = sVmax / l_run;
+            // a split block leaves its unnormalized O, running max and row sum
+            // (in units where O / l is the output) for the merge kernel
+            float* prow = split ? a.part + ((size_t)piece * 256 + qi * 128 + r) * kPartialFloats
+                                : nullptr;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t ov[32];
                 __syncwarp();                  // converged for the collective load
                 tmem_ld32(tO + 32 * q, ov);
                 tmem_wait_ld();
-                if (rvalid) {
+                if (rvalid && split) {
+                    float4* dst = reinterpret_cast<float4*>(prow + 32 * q);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        dst[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                                             __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+                } else if (rvalid) {
                     const size_t o = ((size_t)row * H + h) * kHeadDim + 32 * q;
                     if (a.o_f32) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.O) + o);
@@ -439,6 +470,10 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                     }
                 }
             }
+            if (rvalid && split) {
+                prow[128] = m_run;
+                prow[129] = l_run / sVmax;
+            }
         }
     } else if (warp >= kDequantWarp0) {
         // ------------------------------------------------------------ de-quantize
@@ -451,9 +486,10 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
             uint4 kc[4], vc[4];
             uint2 ks, vs;
         };
-        auto load_row = [&](int tt, int row, Packed& pk) {
-            const int ci = tt / tiles_per_chunk;
-            const int key = (tt - ci * tiles_per_chunk) * kKeysW + row;
+        auto load_row = [&](int tt, int row, Packed& pk) {     // tt: this CTA's tile
+            const int gt = t_begin + tt;
+            const int ci = gt / tiles_per_chunk;
+            const int key = (gt - ci * tiles_per_chunk) * kKeysW + row;
             if (tt < ntiles && key < T_c) {
                 const WsChunk& cp = a.chunk[ci];
                 const size_t rowi = (size_t)h * T_c + key;
@@ -571,7 +607,97 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
     }
 }
 
+// Merge of a split query block: per row, M = max m_q, O = sum 2^(m_q - M) O_q /
+// sum 2^(m_q - M) l_q over its key ranges q.  One warp per row, four outputs
+// per lane.
+__global__ void __launch_bounds__(256) attention_merge_kernel(const float* part, int n_full,
+                                                              int n_tail, int n_split,
+                                                              int pairs_per_head, int T_q, int H,
+                                                              void* O, int o_f32) {
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= n_tail * 256) return;
+    const int tp = w >> 8, rr = w & 255;
+    const int pair = n_full + tp;
+    const int h = pair / pairs_per_head;
+    const int row = (pair - h * pairs_per_head) * 256 + rr;
+    if (row >= T_q) return;
+    const float* base = part + ((size_t)tp * n_split * 256 + rr) * kPartialFloats;
+    const size_t stride = (size_t)256 * kPartialFloats;
+    float M = -INFINITY;
+    for (int q = 0; q < n_split; ++q) M = fmaxf(M, base[q * stride + 128]);
+    float L = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int q = 0; q < n_split; ++q) {
+        const float* pq = base + q * stride;
+        const float wq = exp2f(pq[128] - M);
+        L = fmaf(wq, pq[129], L);
+        const float4 o = reinterpret_cast<const float4*>(pq)[lane];
+        acc.x = fmaf(wq, o.x, acc.x);
+        acc.y = fmaf(wq, o.y, acc.y);
+        acc.z = fmaf(wq, o.z, acc.z);
+        acc.w = fmaf(wq, o.w, acc.w);
+    }
+    const float inv = 1.0f / L;
+    const size_t o = ((size_t)row * H + h) * kHeadDim + 4 * lane;
+    if (o_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(O) + o) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(O) + o) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
+}
+
+int g_sm_count[64];     // multiprocessor count per device ordinal (0 = not yet known)
+
 }  // namespace
+
+// The grid: 256-row query blocks (both tiles of a CTA belong to one head),
+// whole blocks in full waves of one CTA per SM; the blocks left over for a
+// last, partial wave are each split into n_split key ranges, with n_split
+// chosen so that the split pieces finish in the fewest rounds per piece
+// length (ties: fewer pieces), bounded by kMaxSplit, by the key tiles and by
+// the workspace's room for partial results.
+AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs) {
+    AttnPlan p;
+    p.pairs_per_head = (T_q + 255) / 256;
+    p.n_pairs = H * p.pairs_per_head;
+    p.n_full = p.n_pairs;
+    p.n_tail = 0;
+    p.n_split = 1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return p;
+    if (g_sm_count[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            sms <= 0)
+            return p;
+        g_sm_count[dev] = sms;
+    }
+    const int G = g_sm_count[dev];
+    const int n_full = (p.n_pairs / G) * G;
+    const int n_tail = p.n_pairs - n_full;
+    const int ntiles = n_chunks * ((T_c + kKeysW - 1) / kKeysW);
+    if (n_tail == 0 || (size_t)n_tail > tail_capacity_pairs) return p;
+    int best_s = 1;
+    double best = 1.0;                        // rounds x piece length of the unsplit tail
+    for (int sp = 2; sp <= kMaxSplit && sp <= ntiles; ++sp) {
+        const double cost = (double)((n_tail * sp + G - 1) / G) / sp;
+        if (cost < best - 1e-9) {
+            best = cost;
+            best_s = sp;
+        }
+    }
+    if (best_s > 1) {
+        p.n_full = n_full;
+        p.n_tail = n_tail;
+        p.n_split = best_s;
+    }
+    return p;
+}
 
 nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                    int H, const void* Q, int T_q, void* O, int o_dtype,
@@ -583,6 +709,8 @@ nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunk
             return NVFP4KV_ERR_CUDA;
         configured = true;
     }
+    const WsLayout L = ws_layout(T_c, H);
+    const AttnPlan plan = attention_plan(n_chunks, T_c, H, T_q, L.apart_pairs);
     WsArgs a;
     for (int i = 0; i < n_chunks; ++i) {
         a.chunk[i].k_codes = chunks[i].k_codes;
@@ -601,9 +729,21 @@ nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunk
     a.o_f32 = o_dtype == NVFP4KV_F32 ? 1 : 0;
     a.scale_log2 = softmax_scale * kLog2eW;
     a.ctl = static_cast<Control*>(ws);
-    dim3 grid((T_q + 255) / 256, H);
+    a.pairs_per_head = plan.pairs_per_head;
+    a.n_full = plan.n_full;
+    a.n_split = plan.n_split;
+    a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.apart);
+    const int grid = plan.n_full + plan.n_tail * plan.n_split;
     attention_ws_kernel<<<grid, kThreadsW, kSmemW, stream>>>(a);
-    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
+    if (plan.n_tail > 0) {
+        const int warps = plan.n_tail * 256;
+        attention_merge_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(
+            a.part, plan.n_full, plan.n_tail, plan.n_split, plan.pairs_per_head, T_q, H, O,
+            a.o_f32);
+        if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
+    }
+    return NVFP4KV_OK;
 }
 
 }  // namespace nvfp4kv

@@ -14,14 +14,25 @@ constexpr int kHeadDimSupported = 128;   // head dimension d the kernels support
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Attention work split (see launch_attention_ws): the 256-row query blocks
+// that do not fill a whole wave of CTAs are split into up to kMaxSplit key
+// ranges, whose partial results (per row: 128 fp32 outputs, the running max
+// and the row sum) go to the workspace and are merged by a second kernel.
+constexpr int kMaxTailPairs = 160;   // more than one wave never remains
+constexpr int kMaxSplit = 8;
+constexpr int kPartialFloats = 132;  // per row: O[128], m, l, 2 pad (16-byte rows)
+
 // Workspace layout for chunks of T tokens and H heads (d = 128):
 //   [0, 256)  Control (status word, grid barrier)
 //   psum      float    [nseg][H*d]  per-segment column sums of K
 //   pmin/pmax bf16     [nseg][H*d]  per-segment column min / max of K
 //   kpart     float    [kMaxGrid]   per-CTA max |K - mean|
 //   vpart     float    [kMaxGrid]   per-CTA max |V|
+//   (the quantizer uses the workspace up to here: quant_total)
+//   apart     float    [tail pairs * kMaxSplit][256][132]  attention partials,
+//             sized for up to T query rows
 struct WsLayout {
-    size_t psum, pmin, pmax, kpart, vpart, total;
+    size_t psum, pmin, pmax, kpart, vpart, quant_total, apart, apart_pairs, total;
 };
 
 inline WsLayout ws_layout(int T, int H) {
@@ -34,9 +45,21 @@ inline WsLayout ws_layout(int T, int H) {
     L.pmax = off;  off += align256(nseg * HD * 2);
     L.kpart = off; off += align256(kMaxGrid * 4);
     L.vpart = off; off += align256(kMaxGrid * 4);
+    L.quant_total = off;
+    const size_t pairs = (size_t)H * (((size_t)T + 255) / 256);
+    L.apart_pairs = pairs < (size_t)kMaxTailPairs ? pairs : (size_t)kMaxTailPairs;
+    L.apart = off; off += align256(L.apart_pairs * kMaxSplit * 256 * kPartialFloats * 4);
     L.total = off;
     return L;
 }
+
+// How one attention call is laid out on the GPU: n_full whole 256-row query
+// blocks, then n_tail blocks each split into n_split key ranges (n_split = 1:
+// no split, no second kernel).
+struct AttnPlan {
+    int pairs_per_head, n_pairs, n_full, n_tail, n_split;
+};
+AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs);
 
 nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
                                const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream);

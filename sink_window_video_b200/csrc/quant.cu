@@ -775,7 +775,7 @@ extern "C" nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const vo
     if ((mis & 15u) != 0 || (reinterpret_cast<uintptr_t>(out->tensor_scales) & 7u) != 0)
         return NVFP4KV_ERR_ALIGNMENT;
     // the chunk's scratch must fit the compiled-in array
-    if (ws_layout(T_c, H).total > kStaticScratchBytes) return NVFP4KV_ERR_CAPACITY;
+    if (ws_layout(T_c, H).quant_total > kStaticScratchBytes) return NVFP4KV_ERR_CAPACITY;
 
     int dev = 0, major = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4KV_ERR_CUDA;
