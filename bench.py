@@ -52,9 +52,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source it was taken on: a changed source reports null until it is captured again.
 NCU_TRAFFIC = {
     "attention": ("sink_window_video_b200/csrc/attention_ws.cu",
-                  "7c92672a848293abc612987a15e780aa6d40d7dbf4c805bc1b65ef10239375fb", 194599168),
+                  "bb9f84ee22bbdd150b5ed2785787659da5f717cef4d6a9874b87fd91ae2b9be7", 225773824),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
-                 "9e3baa03cec1462f4f474203a0edd716f6f142c9c535cce06c4e93141d5594d2", 133928960),
+                 "8c313008b89b811449016aa51c0c8d49d2a1c6a635c3f210927caccf8c5620b2", 97300224),
 }
 
 
@@ -163,13 +163,21 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(x, world):
+    """The maximum of x over all ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(work_per_step_per_rank, steps, world, ms_max):
+    """Aggregate throughput of a weak-scaling run: every rank does the same work
+    per step; the job takes the slowest rank's time."""
+    return work_per_step_per_rank * steps * world / (ms_max / 1e3)
 
 
 def barrier(world):
@@ -489,7 +497,7 @@ def main():
     peaks, peak_src = load_peaks()
     if rank == 0:
         K = args.steps
-        value = attn_flops() * K * world / (r["ms_total"] / 1e3) / 1e12
+        value = whole_job_rate(attn_flops(), K, world, r["ms_total"]) / 1e12
         attn_tf = attn_flops() / (r["ms_attn"] / 1e3) / 1e12
         quant_gbs = quant_bytes() / (r["ms_quant"] / 1e3) / 1e9
         tpeak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])

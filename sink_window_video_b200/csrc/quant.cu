@@ -223,6 +223,20 @@ __device__ __forceinline__ float max_abs8(const float2* x) {
     return fmaxf(d, fabsf(x[3].y));
 }
 
+// Two bf16 (one word, element 2j low) widened exactly and added to an fp32
+// pair, one rounding each: RN(x + c), as two mixed-precision adds on the FMA
+// pipe (no separate unpacking).
+__device__ __forceinline__ float2 bf16x2_add_f32x2(uint32_t w, float2 c) {
+    float lo, hi;
+    asm("{.reg .b16 l, h;\n"
+        "mov.b32 {l, h}, %2;\n"
+        "add.rn.f32.bf16 %0, l, %3;\n"
+        "add.rn.f32.bf16 %1, h, %4;}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(w), "f"(c.x), "f"(c.y));
+    return make_float2(lo, hi);
+}
+
 // f16 -> f32 (exact) as a mixed-precision add of -0: a full-rate FMA-pipe
 // operation, where cvt.f32.f16 issues at half rate.
 __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h2) {
@@ -372,10 +386,7 @@ __device__ void encode_unit(const QuantArgs& a, QuantShared& sh, bool isK, int h
         {
             const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                x[j] = __fadd2_rn(make_float2(__uint_as_float(u[j] << 16),
-                                              __uint_as_float(u[j] & 0xFFFF0000u)),
-                                  nmu[j]);                          // RN(K - mean), or V
+            for (int j = 0; j < 4; ++j) x[j] = bf16x2_add_f32x2(u[j], nmu[j]);   // RN(K - mean), or V
         }
         const float ah = max_abs8(x);
         const float ab = fmaxf(ah, __shfl_xor_sync(0xFFFFFFFFu, ah, 1));
