@@ -62,6 +62,9 @@ def lib():
                                            ctypes.c_double, vp]
         L.oracle_chunk_payload_bytes.restype = sz
         L.oracle_chunk_payload_bytes.argtypes = [i32, i32, i32]
+        L.oracle_quantize_matrix.restype = i32
+        L.oracle_quantize_matrix.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+        L.oracle_dequantize_matrix.argtypes = [vp, vp, f32, i32, i32, i32, vp]
         L.oracle_set_threads.argtypes = [i32]
         L.oracle_get_threads.restype = i32
         _lib = L
@@ -176,6 +179,35 @@ def dequantize_chunk(q):
     Kh = dequantize_tensor(q["k_codes"], q["k_scales"], q["k_mean"], q["s_k"], T, H, d)
     Vh = dequantize_tensor(q["v_codes"], q["v_scales"], None, q["s_v"], T, H, d)
     return Kh, Vh
+
+
+MATRIX_1D, MATRIX_2D = 1, 2
+
+
+def quantize_matrix(X: np.ndarray, mode: int):
+    """NVFP4 quantization of a bf16 matrix X [M, N] with Four-Over-Six: mode 1
+    (activations) 16-element row blocks, mode 2 (weights) 16 x 16 tiles.
+    Returns dict codes [M, N/2], scales ([M, N/16] or [M/16, N/16]), s, choice."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    M, N = X.shape
+    brows = M if mode == MATRIX_1D else M // 16
+    codes = np.zeros((M, N // 2), np.uint8)
+    scales = np.zeros((brows, N // 16), np.uint8)
+    choice = np.zeros((brows, N // 16), np.uint8)
+    s = np.zeros(1, np.float32)
+    if lib().oracle_quantize_matrix(_ptr(X), M, N, mode, _ptr(codes), _ptr(scales), _ptr(s),
+                                    _ptr(choice)) != 0:
+        raise ValueError(f"shape {X.shape} is not tiled by mode {mode}")
+    return dict(codes=codes, scales=scales, s=float(s[0]), choice=choice)
+
+
+def dequantize_matrix(q: dict, mode: int) -> np.ndarray:
+    M, N2 = q["codes"].shape
+    out = np.zeros((M, 2 * N2), np.float32)
+    lib().oracle_dequantize_matrix(_ptr(np.ascontiguousarray(q["codes"])),
+                                   _ptr(np.ascontiguousarray(q["scales"])), q["s"], M, 2 * N2,
+                                   mode, _ptr(out))
+    return out
 
 
 def payload_bytes(T, H, d) -> int:

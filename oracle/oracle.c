@@ -279,6 +279,109 @@ void oracle_quantize_tensor(const uint16_t* X, int T, int H, int d, float* mean,
     free(Xs);
 }
 
+/*
+ * NVFP4 quantization of a weight or activation matrix with Four-Over-Six
+ * ([DR] Method > 训练基础设施: NVFP4 weights and activations -- E2M1 values,
+ * FP8 E4M3 block scales, an FP32 tensor scale, the block scale searched over
+ * targets 6 and 4; the block shape follows the operand: 1D blocks along a row
+ * for activations, 2D 16 x 16 blocks for weights).
+ *   X: [M][N] bf16, row-major; N a multiple of 16 (and M too for 2D).
+ *   mode 1 (activations): a block is 16 consecutive elements of a row;
+ *          scales [M][N/16].
+ *   mode 2 (weights): a block is a 16 x 16 tile; scales [M/16][N/16].
+ *   s = max|X| / (6*448)  (1 if X is all zero).
+ * Per block and target m: sb = E4M3(amax / (m*s)), D = decode(sb) * s,
+ * q_i = E2M1(x_i / D) (+0 when D == 0), e_i = x_i - decode(q_i)*D.  The block
+ * error, in fp32: each 16-element row segment of the block gives
+ * (e_0^2 + .. + e_7^2) + (e_8^2 + .. + e_15^2) (each half left to right), and
+ * the segments are added in increasing row order -- the same as the KV blocks
+ * for 1D.  Keep 4 only if its error is strictly lower.
+ * Codes [M][N/2], element 2j of a row in the low nibble of byte j.
+ * choice (optional): [number of blocks], 1 where target 4 was kept.
+ * Returns 0, or -1 for shapes the mode does not tile.
+ */
+static float matrix_segment(const float* x, float D, uint8_t* q) {
+    float lo = 0.0f, hi = 0.0f;
+    for (int i = 0; i < BLOCK; ++i) {
+        q[i] = (D > 0.0f) ? oracle_e2m1_encode(x[i] / D) : 0;
+        float e = x[i] - oracle_e2m1_decode(q[i]) * D;
+        float e2 = e * e;
+        if (i < BLOCK / 2) lo = (i == 0) ? e2 : lo + e2;
+        else               hi = (i == BLOCK / 2) ? e2 : hi + e2;
+    }
+    return lo + hi;
+}
+
+int oracle_quantize_matrix(const uint16_t* X, int M, int N, int mode, uint8_t* codes,
+                           uint8_t* scales, float* tensor_scale, uint8_t* choice) {
+    if (M <= 0 || N <= 0 || N % BLOCK != 0 || (mode == 2 && M % BLOCK != 0) ||
+        (mode != 1 && mode != 2))
+        return -1;
+    size_t n = (size_t)M * N;
+    float* Xf = (float*)malloc(n * sizeof(float));
+    float A = 0.0f;
+    #pragma omp parallel for schedule(static) reduction(max:A)
+    for (long long i = 0; i < (long long)n; ++i) {
+        Xf[i] = oracle_bf16_to_f32(X[i]);
+        float av = fabsf(Xf[i]);
+        if (av > A) A = av;
+    }
+    float s = (A > 0.0f) ? A / TENSOR_SCALE_DIV : 1.0f;
+    *tensor_scale = s;
+    const int rows = (mode == 1) ? 1 : BLOCK;            /* row segments per block */
+    const int brows = M / rows, bcols = N / BLOCK;
+    #pragma omp parallel for schedule(static)
+    for (int br = 0; br < brows; ++br)
+        for (int bc = 0; bc < bcols; ++bc) {
+            float amax = 0.0f;
+            for (int r = 0; r < rows; ++r)
+                for (int i = 0; i < BLOCK; ++i) {
+                    float av = fabsf(Xf[(size_t)(br * rows + r) * N + bc * BLOCK + i]);
+                    if (av > amax) amax = av;
+                }
+            uint8_t sb[2], q[2][BLOCK * BLOCK];
+            float err[2];
+            const float targets[2] = {6.0f, 4.0f};
+            for (int k = 0; k < 2; ++k) {
+                float ratio = amax / (targets[k] * s);
+                sb[k] = oracle_e4m3_encode(ratio);
+                float D = oracle_e4m3_decode(sb[k]) * s;
+                float E = 0.0f;
+                for (int r = 0; r < rows; ++r) {
+                    float seg = matrix_segment(Xf + (size_t)(br * rows + r) * N + bc * BLOCK, D,
+                                               q[k] + r * BLOCK);
+                    E = (r == 0) ? seg : E + seg;
+                }
+                err[k] = E;
+            }
+            int keep4 = err[1] < err[0];            /* a tie keeps target 6 */
+            scales[(size_t)br * bcols + bc] = sb[keep4];
+            if (choice) choice[(size_t)br * bcols + bc] = (uint8_t)keep4;
+            for (int r = 0; r < rows; ++r) {
+                uint8_t* out = codes + (size_t)(br * rows + r) * (N / 2) + bc * (BLOCK / 2);
+                const uint8_t* qq = q[keep4] + r * BLOCK;
+                for (int j = 0; j < BLOCK / 2; ++j)
+                    out[j] = (uint8_t)((qq[2 * j] & 15u) | ((qq[2 * j + 1] & 15u) << 4));
+            }
+        }
+    free(Xf);
+    return 0;
+}
+
+/* De-quantize a matrix quantized by oracle_quantize_matrix: fp32 [M][N],
+ * x_hat = decode(q) * (decode(sb) * s). */
+void oracle_dequantize_matrix(const uint8_t* codes, const uint8_t* scales, float s, int M,
+                              int N, int mode, float* out) {
+    const int rows = (mode == 1) ? 1 : BLOCK;
+    for (int r = 0; r < M; ++r)
+        for (int c = 0; c < N; ++c) {
+            uint8_t byte = codes[(size_t)r * (N / 2) + c / 2];
+            uint8_t q = (c & 1) ? (byte >> 4) : (byte & 15u);
+            float D = oracle_e4m3_decode(scales[(size_t)(r / rows) * (N / BLOCK) + c / BLOCK]) * s;
+            out[(size_t)r * N + c] = oracle_e2m1_decode(q) * D;
+        }
+}
+
 /* Both tensors of a chunk: K with smoothing, V without. */
 void oracle_quantize_chunk(const uint16_t* K, const uint16_t* V, int T, int H, int d,
                            uint8_t* k_codes, uint8_t* k_scales,

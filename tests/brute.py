@@ -130,3 +130,40 @@ def unpack_codes(packed: np.ndarray) -> np.ndarray:
     out[..., 0::2] = p & 15
     out[..., 1::2] = p >> 4
     return out
+
+
+def four_over_six_tiles(x: np.ndarray, s: np.float32):
+    """Brute-force Four-Over-Six over 16 x 16 tiles x [ntiles, 16, 16] (float32):
+    one scale per tile from the tile max; codes as in four_over_six_blocks; the
+    tile error adds, row by row in increasing row order, each row's
+    (elements 0..7) + (elements 8..15) sum.  Returns (codes [ntiles,16,16],
+    scale bytes [ntiles], keep4 [ntiles])."""
+    x = np.ascontiguousarray(x, np.float32)
+    s = np.float32(s)
+    nt = x.shape[0]
+    amax = np.abs(x).reshape(nt, -1).max(axis=1)
+    res = {}
+    for m in (6, 4):
+        ratio = amax / (np.float32(m) * s)
+        sb = brute_e4m3(ratio.astype(np.float32))
+        D = e4m3_value(sb) * s
+        Dc = np.where(D > 0, D, np.float32(1))[:, None, None]
+        y = (x / Dc).astype(np.float32)
+        q = brute_e2m1(y.reshape(-1)).reshape(x.shape)
+        q = np.where((D > 0)[:, None, None], q, 0).astype(np.uint8)
+        e = x - e2m1_value(q) * D[:, None, None]
+        e2 = (e * e).astype(np.float32)
+        lo = e2[:, :, 0].copy()
+        hi = e2[:, :, 8].copy()
+        for i in range(1, 8):
+            lo = (lo + e2[:, :, i]).astype(np.float32)
+            hi = (hi + e2[:, :, 8 + i]).astype(np.float32)
+        seg = (lo + hi).astype(np.float32)          # [ntiles, 16 rows]
+        E = seg[:, 0].copy()
+        for r in range(1, 16):
+            E = (E + seg[:, r]).astype(np.float32)
+        res[m] = (q, sb, E)
+    keep4 = res[4][2] < res[6][2]
+    codes = np.where(keep4[:, None, None], res[4][0], res[6][0])
+    sbytes = np.where(keep4, res[4][1], res[6][1])
+    return codes.astype(np.uint8), sbytes.astype(np.uint8), keep4
