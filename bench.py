@@ -314,13 +314,54 @@ def run_ours(args, rank, world, local):
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
 
+    matrix = run_matrix_quant(swv, pool, stream) if not args.no_matrix else None
+
     rollouts = None
     if not args.no_rollout:
         rollouts = [run_rollout(swv, cfg, pool, O, stream, world) for cfg in ROLLOUTS]
 
     return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
-                e2e_ms=e2e_ms, rollouts=rollouts,
+                e2e_ms=e2e_ms, rollouts=rollouts, matrix=matrix,
                 attn_launches=swv.attention_launches(len(cache.keyset(0)), T, H, T))
+
+
+# ------------------------------------------------------------------ weights / activations
+
+MATRIX_SHAPES = (("activations [7040, 3072] bf16, 16-element row blocks", 1, 7040, 3072),
+                 ("weights [3072, 3072] bf16, 16 x 16 tiles", 2, 3072, 3072))
+
+
+def run_matrix_quant(swv, pool, stream, launches=40):
+    """NVFP4 quantization of the 5B DiT's activation and weight shapes; inputs
+    rotate over 8 distinct device tensors (the pool's K and V, 151-346 MB,
+    larger than L2), CUDA events around each launch."""
+    import torch
+    peaks, src = load_peaks()
+    hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    ws = swv.new_matrix_workspace()
+    res = []
+    for name, mode, M, N in MATRIX_SHAPES:
+        srcs = [t.view(-1)[:M * N].view(M, N) for s3 in pool for t in s3[:2]]
+        out = swv.MatrixBuffer(M, N, mode)
+        for i in range(3):
+            swv.quantize_matrix(srcs[i % len(srcs)], out, ws)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(launches)]
+        torch.cuda.synchronize()
+        for i, (e0, e1) in enumerate(ev):
+            e0.record(stream)
+            swv.quantize_matrix(srcs[i % len(srcs)], out, ws)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        if swv.workspace_status(ws) != swv.OK:
+            raise RuntimeError("device status not OK after the matrix quantizer")
+        us = 1e3 * sum(e0.elapsed_time(e1) for e0, e1 in ev) / launches
+        nbytes = 2 * M * N + M * N // 2 + (M * N // 16 if mode == 1 else M * N // 256) + 4
+        gbs = nbytes / (us / 1e6) / 1e9
+        res.append({"workload": name, "us_per_launch": us, "bytes_per_launch": nbytes,
+                    "achieved": gbs, "unit": "GB/s", "peak": hpeak, "frac": gbs / hpeak,
+                    "bound": "hbm", "peak_source": f"{src} hbm"})
+    return res
 
 
 # ------------------------------------------------------------------ rollouts
@@ -483,6 +524,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rollout", action="store_true")
+    ap.add_argument("--no-matrix", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -532,6 +574,8 @@ def main():
                            "d2h_bytes_per_step": n * 2, "ms_per_step": r["e2e_ms"]}
         if r["rollouts"] is not None:
             line["rollouts"] = r["rollouts"]
+        if r["matrix"] is not None:
+            line["matrix_quantize"] = r["matrix"]
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = OracleSample(rows=args.ref_rows).baseline()
         print(json.dumps(line))

@@ -166,6 +166,43 @@ nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const void* V, int 
                                               int d, const nvfp4kv_chunk_view* out,
                                               nvfp4kv_stream_t stream);
 
+/* ------------------------------------------------------------------ weights / activations */
+
+/* Block shape of nvfp4kv_quantize_matrix. */
+typedef enum {
+    NVFP4KV_BLOCKS_1D = 1,   /* 16 consecutive elements of a row (activations) */
+    NVFP4KV_TILES_2D = 2     /* 16 x 16 tiles (weights) */
+} nvfp4kv_block_shape;
+
+/* Bytes of the workspace of nvfp4kv_quantize_matrix (any shape). */
+size_t nvfp4kv_matrix_workspace_bytes(void);
+
+/*
+ * NVFP4 quantization of a weight or activation matrix with Four-Over-Six
+ * (DeepRead page, Method > 训练基础设施: NVFP4 weights and activations, E2M1
+ * values under FP8 E4M3 block scales and one FP32 tensor scale, each block's
+ * scale searched over targets 6 and 4; the block shape follows the operand --
+ * 1D for activations, 2D 16 x 16 for weights).
+ *   X: [M][N] bf16 row-major, device, 16-byte aligned; N a multiple of 16
+ *      (and M too for NVFP4KV_TILES_2D), else NVFP4KV_ERR_UNSUPPORTED.
+ *   s = max|X| / (6*448) (1 if all zero), written to *tensor_scale (device float).
+ *   Per block and target m in {6, 4}: sb = E4M3(amax / (m*s)), D = decode(sb)*s,
+ *   codes E2M1(x / D) (+0 when D == 0); the block error adds, row segment by
+ *   row segment in increasing row order, (e_0^2 + .. + e_7^2) + (e_8^2 + ..
+ *   + e_15^2); the 4-encoding is kept only if its error is strictly lower.
+ *   codes:  [M][N/2] bytes (device, 16-byte aligned), element 2j of a row in
+ *           the low nibble of byte j;
+ *   scales: [M][N/16] (1D) or [M/16][N/16] (2D) E4M3 bytes (device).
+ *   ws: device, 256-byte aligned, nvfp4kv_matrix_workspace_bytes() long,
+ *       initialized once with nvfp4kv_workspace_init (its status word reports
+ *       a grid barrier that gave up, see nvfp4kv_workspace_status).
+ * Results are bit-identical to the definition above.  The caller owns all
+ * memory; X and the outputs must not overlap.
+ */
+nvfp4kv_status nvfp4kv_quantize_matrix(const void* X, int M, int N, int mode, void* codes,
+                                       void* scales, float* tensor_scale, void* ws,
+                                       nvfp4kv_stream_t stream);
+
 /*
  * De-quantize a chunk back to [T_c][H][d] (device): x = decode(q) *
  * (decode(scale) * s), plus mean for K, each step one fp32 operation.

@@ -69,6 +69,8 @@ def load():
         "nvfp4kv_dequantize": (st, [cv, i32, i32, i32, vp, vp, i32, vp]),
         "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp]),
         "nvfp4kv_attention_launches": (i32, [i32, i32, i32, i32, i32]),
+        "nvfp4kv_matrix_workspace_bytes": (sz, []),
+        "nvfp4kv_quantize_matrix": (st, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
         "kvcache_pool_bytes": (sz, [cfgp]),
         "kvcache_create": (st, [cfgp, vp, vp, ctypes.POINTER(vp)]),
         "kvcache_destroy": (None, [vp]),
@@ -131,6 +133,44 @@ def version() -> str:
 
 def chunk_bytes(T_c, H, d=HEAD_DIM) -> int:
     return int(load().nvfp4kv_chunk_bytes(T_c, H, d))
+
+
+BLOCKS_1D, TILES_2D = 1, 2
+
+
+class MatrixBuffer:
+    """Device buffers of a quantized [M, N] matrix: codes [M, N/2] (uint8),
+    scales ([M, N/16] for 1D blocks, [M/16, N/16] for 2D tiles), tensor scale."""
+
+    def __init__(self, M, N, mode, device="cuda"):
+        import torch
+        self.M, self.N, self.mode = M, N, mode
+        brows = M if mode == BLOCKS_1D else M // 16
+        self.codes = torch.zeros((M, N // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.zeros((brows, N // 16), dtype=torch.uint8, device=device)
+        self.tensor_scale = torch.zeros(1, dtype=torch.float32, device=device)
+
+    def to_host(self):
+        return dict(codes=self.codes.cpu().numpy(), scales=self.scales.cpu().numpy(),
+                    s=float(self.tensor_scale[0].item()))
+
+
+def new_matrix_workspace(device="cuda", stream=None):
+    import torch
+    ws = torch.zeros(int(load().nvfp4kv_matrix_workspace_bytes()), dtype=torch.uint8,
+                     device=device)
+    workspace_init(ws, stream)
+    return ws
+
+
+def quantize_matrix(X, out: "MatrixBuffer", ws, stream=None):
+    """NVFP4 quantization of a bf16 [M, N] matrix with Four-Over-Six (1D row
+    blocks or 2D 16 x 16 tiles, out.mode)."""
+    M, N = X.shape
+    _check(load().nvfp4kv_quantize_matrix(_ptr(X), M, N, out.mode, _ptr(out.codes),
+                                          _ptr(out.scales), _ptr(out.tensor_scale), _ptr(ws),
+                                          _stream(stream)),
+           "nvfp4kv_quantize_matrix")
 
 
 def attention_launches(n_chunks, T_c, H, T_q, d=HEAD_DIM) -> int:

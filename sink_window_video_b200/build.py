@@ -22,6 +22,7 @@ COMMON = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
                  "-I" + INCLUDE, "-I" + CSRC, "--expt-relaxed-constexpr"]
 PER_FILE = {
     "quant.cu": ["-fmad=false"],
+    "matrix_quant.cu": ["-fmad=false"],
 }
 
 

@@ -208,6 +208,24 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
     return launch_quantize(K, V, T_c, H, *out, ws, (cudaStream_t)stream);
 }
 
+size_t nvfp4kv_matrix_workspace_bytes(void) { return matrix_workspace_bytes(); }
+
+nvfp4kv_status nvfp4kv_quantize_matrix(const void* X, int M, int N, int mode, void* codes,
+                                       void* scales, float* tensor_scale, void* ws,
+                                       nvfp4kv_stream_t stream) {
+    if (!X || !codes || !scales || !tensor_scale || !ws || M <= 0 || N <= 0 ||
+        (mode != NVFP4KV_BLOCKS_1D && mode != NVFP4KV_TILES_2D) || M > (1 << 24) ||
+        N > (1 << 24) || (long long)M * N > (1ll << 34))
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (N % 16 != 0 || (mode == NVFP4KV_TILES_2D && M % 16 != 0)) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned16(X) || !aligned16(codes) || !aligned256(ws) ||
+        (reinterpret_cast<uintptr_t>(tensor_scale) & 3u) != 0)
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_quantize_matrix(X, M, N, mode, codes, scales, tensor_scale, ws,
+                                  (cudaStream_t)stream);
+}
+
 nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, int d,
                                   void* K_out, void* V_out, int out_dtype,
                                   nvfp4kv_stream_t stream) {

@@ -64,6 +64,13 @@ AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capac
 nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
                                const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream);
 
+// Weight / activation quantizer (matrix_quant.cu): workspace = control block +
+// per-CTA partial maxima.
+size_t matrix_workspace_bytes();
+nvfp4kv_status launch_quantize_matrix(const void* X, int M, int N, int mode, void* codes,
+                                      void* scales, float* tensor_scale, void* ws,
+                                      cudaStream_t stream);
+
 nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, void* K_out,
                                  void* V_out, int out_dtype, cudaStream_t stream);
 

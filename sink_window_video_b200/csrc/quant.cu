@@ -33,6 +33,7 @@
 // and tensor scales are bit-identical to the definition.
 #include "common.cuh"
 #include "kernels.h"
+#include "nvfp4_encode.cuh"
 
 namespace nvfp4kv {
 namespace {
@@ -42,12 +43,6 @@ constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kEncTokens = 8;          // tokens per encoding unit (one warp)
 constexpr int kFinCols = 32;           // columns per finalize block (one per lane)
 constexpr int kFinSegs = 120;          // segments staged per finalize pass (5 per warp)
-// Markstein's quotient is correctly rounded when no step underflows: the
-// tensor scale and the block max are kept above these bounds, else the
-// quotient is an IEEE division.
-constexpr float kFastMinScale = 0x1p-90f;
-constexpr float kFastMinBlockMax = 0x1p-100f;
-
 struct QuantArgs {
     const uint4* K;
     const uint4* V;
@@ -94,26 +89,6 @@ __device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) {
 }
 __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
     return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// L2 eviction policies: inputs read twice are kept (evict_last) on the first
-// read and released (evict_first) on the second.
-__device__ __forceinline__ uint64_t policy_keep() {
-    uint64_t p;
-    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ uint64_t policy_release() {
-    uint64_t p;
-    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ uint4 ld_hint(const uint4* p, uint64_t pol) {
-    uint4 r;
-    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p), "l"(pol));
-    return r;
 }
 
 // The tensor scale from the per-CTA partial maxima, and the decode table.
@@ -215,136 +190,6 @@ __device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
 
 // ---------------------------------------------------------------- encoding
 
-__device__ __forceinline__ float max_abs8(const float2* x) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(x[0].x)), "f"(fabsf(x[0].y)), "f"(fabsf(x[1].x)));
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(d), "f"(fabsf(x[1].y)), "f"(fabsf(x[2].x)));
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(d), "f"(fabsf(x[2].y)), "f"(fabsf(x[3].x)));
-    return fmaxf(d, fabsf(x[3].y));
-}
-
-// Two bf16 (one word, element 2j low) widened exactly and added to an fp32
-// pair, one rounding each: RN(x + c), as two mixed-precision adds on the FMA
-// pipe (no separate unpacking).
-__device__ __forceinline__ float2 bf16x2_add_f32x2(uint32_t w, float2 c) {
-    float lo, hi;
-    asm("{.reg .b16 l, h;\n"
-        "mov.b32 {l, h}, %2;\n"
-        "add.rn.f32.bf16 %0, l, %3;\n"
-        "add.rn.f32.bf16 %1, h, %4;}"
-        : "=f"(lo), "=f"(hi)
-        : "r"(w), "f"(c.x), "f"(c.y));
-    return make_float2(lo, hi);
-}
-
-// f16 -> f32 (exact) as a mixed-precision add of -0: a full-rate FMA-pipe
-// operation, where cvt.f32.f16 issues at half rate.
-__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h2) {
-    float lo, hi;
-    asm("{.reg .b16 l, h;\n"
-        "mov.b32 {l, h}, %2;\n"
-        "add.rn.f32.f16 %0, l, 0f80000000;\n"
-        "add.rn.f32.f16 %1, h, 0f80000000;}"
-        : "=f"(lo), "=f"(hi)
-        : "r"(h2));
-    return make_float2(lo, hi);
-}
-
-// Four fp32 pairs -> the packed E2M1 codes (byte j = elements 2j, 2j+1) and
-// their decoded values as four f16x2, from the same conversion bytes.
-__device__ __forceinline__ uint32_t cvt_e2m1x8_dec(const float* v, uint32_t* h) {
-    uint32_t r;
-    asm("{\n"
-        ".reg .b8 b0, b1, b2, b3;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n"
-        "cvt.rn.f16x2.e2m1x2 %1, b0;\n"
-        "cvt.rn.f16x2.e2m1x2 %2, b1;\n"
-        "cvt.rn.f16x2.e2m1x2 %3, b2;\n"
-        "cvt.rn.f16x2.e2m1x2 %4, b3;\n"
-        "mov.b32 %0, {b0, b1, b2, b3};\n"
-        "}"
-        : "=r"(r), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
-          "f"(v[7]));
-    return r;
-}
-
-// Eight elements (four pairs) against one candidate step D with r = RN(1/D):
-// packed codes q (byte j = elements 2j, 2j+1) and the sequential sum of the
-// eight squared errors RN(RN(x - RN(decode(q) * D))^2).
-// The quotient is Markstein's, computed for -x / D so that a zero keeps its
-// sign: n0 = RN(x (-r)), e = x + n0 D (exact), n1 = RN(n0 - e r) = -RN(x / D).
-// The codes of -x / D are those of x / D with the sign bits flipped (one XOR
-// for the stored word); their decoded values dq' = -dq give the error
-// directly: RN(x - RN(dq D)) = RN(x + RN(dq' D)).
-// The compiler merges a paired product followed by a paired sum into one
-// fused multiply-add, which would skip the product's rounding; every sum is
-// therefore written as a fused multiply-add whose other factor is 1 held in a
-// run-time value (exact, and not mergeable).
-__device__ __forceinline__ void encode8_fast(const float2* x, float2 Dr, float one, uint32_t& q,
-                                             float& err) {
-    const float2 NR = make_float2(-Dr.y, -Dr.y);
-    const float2 D2 = make_float2(Dr.x, Dr.x);
-    float y[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 n0 = __fmul2_rn(x[j], NR);
-        const float2 e = __ffma2_rn(n0, D2, x[j]);
-        const float2 n1 = __ffma2_rn(e, NR, n0);
-        y[2 * j] = n1.x;
-        y[2 * j + 1] = n1.y;
-    }
-    uint32_t h[4];
-    q = cvt_e2m1x8_dec(y, h) ^ 0x88888888u;
-    const float2 ONE = make_float2(one, one);
-    float acc = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 p = __fmul2_rn(f16x2_to_f32x2(h[j]), D2);      // RN(dq' D) = -RN(dq D)
-        const float2 d = __ffma2_rn(p, ONE, x[j]);                   // RN(x - RN(dq D))
-        const float2 sq = __fmul2_rn(d, d);
-        acc = (j == 0) ? sq.x : __fmaf_rn(sq.x, one, acc);
-        acc = __fmaf_rn(sq.y, one, acc);
-    }
-    err = acc;
-}
-
-// The same with IEEE divisions (tensor scales too small for the fast path);
-// out of line, so the rare path costs no instruction-cache space in the loop.
-struct Enc8 {
-    uint32_t q;
-    float err;
-};
-
-__device__ __noinline__ Enc8 encode8_slow(float x0, float x1, float x2, float x3, float x4,
-                                          float x5, float x6, float x7, float D) {
-    const float x[8] = {x0, x1, x2, x3, x4, x5, x6, x7};
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = D > 0.0f ? __fdiv_rn(x[i], D) : 0.0f;
-    Enc8 r;
-    r.q = cvt_e2m1x8(y);
-    uint32_t h[4];
-    cvt_e2m1x8_to_f16x2(r.q, h);
-    float acc = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float e0 = __fsub_rn(x[2 * j], __fmul_rn(f16lo(h[j]), D));
-        const float e1 = __fsub_rn(x[2 * j + 1], __fmul_rn(f16hi(h[j]), D));
-        acc = (j == 0) ? __fmul_rn(e0, e0) : __fadd_rn(acc, __fmul_rn(e0, e0));
-        acc = __fadd_rn(acc, __fmul_rn(e1, e1));
-    }
-    r.err = acc;
-    return r;
-}
-
-__device__ __noinline__ float2 ratio_slow(float ab, float ms6, float ms4) {
-    return make_float2(__fdiv_rn(ab, ms6), __fdiv_rn(ab, ms4));
-}
-
 // One unit: head h, tokens [t0, t0 + 8) of K (mean subtracted) or V (mean
 // -0: x + (-0) = x exactly, signed zeros included).  Lane = (token parity,
 // 8-channel group); iteration it covers tokens t0 + 2 it + {0, 1}, with the
@@ -432,22 +277,6 @@ __device__ void encode_unit(const QuantArgs& a, QuantShared& sh, bool isK, int h
             *reinterpret_cast<const uint2*>(&sh.sb[warp][lane * 8]);
     }
     __syncwarp();
-}
-
-struct EncodeConsts {
-    float s, ms6, ms4;
-    float2 rm;
-    bool fast;
-};
-
-__device__ __forceinline__ EncodeConsts encode_consts(float s) {
-    EncodeConsts c;
-    c.s = s;
-    c.ms6 = __fmul_rn(6.0f, s);
-    c.ms4 = __fmul_rn(4.0f, s);
-    c.rm = make_float2(__frcp_rn(c.ms6), __frcp_rn(c.ms4));
-    c.fast = s >= kFastMinScale;
-    return c;
 }
 
 // ---------------------------------------------------------------- phase B

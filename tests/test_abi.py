@@ -77,6 +77,13 @@ def test_rejects_bad_arguments_without_device_work(L):
     assert a(arr, 1, 32, 2, 96, FAKE, 32, FAKE, 1, 0.0, FAKE, None) == swv.ERR_UNSUPPORTED
     assert a(arr, 1, 32, 2, 128, FAKE, 32, FAKE, 7, 0.0, FAKE, None) == swv.ERR_INVALID_ARG
     assert L.nvfp4kv_check_formats(9, FAKE, FAKE, 1, None) == swv.ERR_INVALID_ARG
+    m = L.nvfp4kv_quantize_matrix
+    assert m(None, 16, 32, 1, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_INVALID_ARG
+    assert m(FAKE, 16, 32, 3, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_INVALID_ARG
+    assert m(FAKE, 16, 40, 1, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_UNSUPPORTED
+    assert m(FAKE, 24, 32, 2, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_UNSUPPORTED
+    assert m(FAKE + 8, 16, 32, 2, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_ALIGNMENT
+    assert L.nvfp4kv_matrix_workspace_bytes() >= 256
     assert L.nvfp4kv_workspace_init(None, 256, None) == swv.ERR_INVALID_ARG
 
 
