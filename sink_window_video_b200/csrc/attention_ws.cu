@@ -11,13 +11,13 @@
 // into fp16 range.
 //
 // One CTA per SM: a head and 256 query rows (two 128-row tiles Q0, Q1), keys
-// in 128-key tiles.  Warp roles (352 threads; 11 warps keep 168 registers per
+// in 128-key tiles.  Warp roles (384 threads; 12 warps keep 168 registers per
 // thread, registers being split among the four SM sub-partitions):
 //   warps 0-3   softmax of Q0 (thread = row = TMEM lane)
 //   warps 4-7   softmax of Q1
 //   warp 8      tensor memory allocation and the MMA issue (one thread)
-//   warps 9-10  de-quantize K and V tiles (two key rows per thread) into a
-//               2-stage shared-memory ring (128-byte-swizzled: K-major B of
+//   warps 9-11  de-quantize K and V tiles (three row conversions per thread)
+//               into a 2-stage shared-memory ring (128-byte-swizzled: K-major B of
 //               S = Q K^T, MN-major B of P V)
 // (warp w runs on SM sub-partition w mod 4.)
 // Tile size: every tcgen05.mma of M = 128, K = 16 costs about the same issue
@@ -53,7 +53,8 @@ namespace {
 
 constexpr int kKeysW = 128;                 // keys per tile
 constexpr int kStages = 2;                  // de-quantized K/V ring depth
-constexpr int kThreadsW = 352;
+constexpr int kThreadsW = 384;
+constexpr int kDequantWarps = 3;
 constexpr int kMmaWarp = 8;
 constexpr int kDequantWarp0 = 9;
 constexpr uint32_t kColS = 0, kColO = 256, kColsW = 512;
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
     if (tid == 0) {
         sh.abort = 0;
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&sh.kv_full[s]), 64);
+            mbar_init(smem_u32(&sh.kv_full[s]), 32 * kDequantWarps);
             mbar_init(smem_u32(&sh.kv_empty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -477,37 +478,41 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         }
     } else if (warp >= kDequantWarp0) {
         // ------------------------------------------------------------ de-quantize
-        // Each thread converts key rows kl and kl + 64.  A row's codes and
-        // scales for the next tile are loaded right after the row is
-        // converted, so the L2 latency overlaps the rest of the tile period.
-        // Rows past a chunk's end get zero codes and zero scales: exact zeros.
-        const int kl = tid - kDequantWarp0 * 32;           // 0..63
+        // 256 row conversions per tile (128 key rows of K and of V), spread
+        // over the 96 threads of three warps (one per sub-partition 1-3):
+        // thread j takes conversions j, j + 96, j + 192.  A conversion's codes
+        // and scales for the next tile are loaded right after it is done, so
+        // the L2 latency overlaps the rest of the tile period.  Rows past a
+        // chunk's end get zero codes and zero scales: exact zeros.
+        const int j = tid - kDequantWarp0 * 32;             // 0..95
+        constexpr int kJobs = 3;
         struct Packed {
-            uint4 kc[4], vc[4];
-            uint2 ks, vs;
+            uint4 c[4];
+            uint2 s;
         };
-        auto load_row = [&](int tt, int row, Packed& pk) {     // tt: this CTA's tile
+        auto load_row = [&](int tt, int job, Packed& pk) {     // tt: this CTA's tile
+            const int row = job >> 1;
             const int gt = t_begin + tt;
             const int ci = gt / tiles_per_chunk;
             const int key = (gt - ci * tiles_per_chunk) * kKeysW + row;
-            if (tt < ntiles && key < T_c) {
+            if (job < 256 && tt < ntiles && key < T_c) {
                 const WsChunk& cp = a.chunk[ci];
                 const size_t rowi = (size_t)h * T_c + key;
-                const uint4* kp = reinterpret_cast<const uint4*>(cp.k_codes + rowi * 64);
-                const uint4* vp = reinterpret_cast<const uint4*>(cp.v_codes + rowi * 64);
+                const uint8_t* codes = (job & 1) ? cp.v_codes : cp.k_codes;
+                const uint8_t* scales = (job & 1) ? cp.v_scales : cp.k_scales;
+                const uint4* p4 = reinterpret_cast<const uint4*>(codes + rowi * 64);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) { pk.kc[i] = kp[i]; pk.vc[i] = vp[i]; }
-                pk.ks = *reinterpret_cast<const uint2*>(cp.k_scales + rowi * 8);
-                pk.vs = *reinterpret_cast<const uint2*>(cp.v_scales + rowi * 8);
+                for (int i = 0; i < 4; ++i) pk.c[i] = p4[i];
+                pk.s = *reinterpret_cast<const uint2*>(scales + rowi * 8);
             } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pk.kc[i] = pk.vc[i] = make_uint4(0, 0, 0, 0);
-                pk.ks = pk.vs = make_uint2(0, 0);
+                for (int i = 0; i < 4; ++i) pk.c[i] = make_uint4(0, 0, 0, 0);
+                pk.s = make_uint2(0, 0);
             }
         };
-        Packed ra, rb;
-        load_row(0, kl, ra);
-        load_row(0, kl + 64, rb);
+        Packed rj[kJobs];
+#pragma unroll
+        for (int m = 0; m < kJobs; ++m) load_row(0, j + 96 * m, rj[m]);
         for (int t = 0; t < ntiles; ++t) {
             const int st = t % kStages;
             if (t >= kStages) {
@@ -515,14 +520,15 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                                          (uint32_t)(((t / kStages) - 1) & 1), abort, a.ctl, 30u, t);
                 if (!__all_sync(0xFFFFFFFFu, got)) break;
             }
-            uint8_t* kt = Kt + st * kTileB;
-            uint8_t* vt = Vt + st * kTileB;
-            dequant_row_regs(ra.kc, ra.ks, kt, kl);
-            dequant_row_regs(ra.vc, ra.vs, vt, kl);
-            load_row(t + 1, kl, ra);
-            dequant_row_regs(rb.kc, rb.ks, kt, kl + 64);
-            dequant_row_regs(rb.vc, rb.vs, vt, kl + 64);
-            load_row(t + 1, kl + 64, rb);
+#pragma unroll
+            for (int m = 0; m < kJobs; ++m) {
+                const int job = j + 96 * m;
+                if (job < 256) {
+                    uint8_t* tile = ((job & 1) ? Vt : Kt) + st * kTileB;
+                    dequant_row_regs(rj[m].c, rj[m].s, tile, job >> 1);
+                }
+                load_row(t + 1, job, rj[m]);
+            }
             fence_async_smem();
             mbar_arrive(smem_u32(&sh.kv_full[st]));
         }
