@@ -52,7 +52,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source it was taken on: a changed source reports null until it is captured again.
 NCU_TRAFFIC = {
     "attention": ("sink_window_video_b200/csrc/attention_ws.cu",
-                  "bb9f84ee22bbdd150b5ed2785787659da5f717cef4d6a9874b87fd91ae2b9be7", 225773824),
+                  "43b4b027366a454ad09f5f26b6249269c83917684536fd5377be5b4fa8e97927", 224931072),
+    "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
+                  "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
                  "8c313008b89b811449016aa51c0c8d49d2a1c6a635c3f210927caccf8c5620b2", 97300224),
 }
@@ -360,7 +362,8 @@ def run_matrix_quant(swv, pool, stream, launches=40):
         gbs = nbytes / (us / 1e6) / 1e9
         res.append({"workload": name, "us_per_launch": us, "bytes_per_launch": nbytes,
                     "achieved": gbs, "unit": "GB/s", "peak": hpeak, "frac": gbs / hpeak,
-                    "bound": "hbm", "peak_source": f"{src} hbm"})
+                    "bound": "hbm", "peak_source": f"{src} hbm",
+                    "traffic": ncu_traffic("matrix_1d") if mode == 1 else None})
     return res
 
 

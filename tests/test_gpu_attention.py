@@ -155,3 +155,33 @@ def test_empty_keyset_is_an_error(lib):
     with pytest.raises(lib.NvFp4KvError) as e:
         cache.attention(0, Q, O)
     assert e.value.status == lib.ERR_EMPTY_KEYSET
+
+
+@pytest.mark.parametrize("H,T_c,T_q,launches", [(37, 64, 1024, 1), (2, 64, 2048, 1), (3, 600, 500, 2)],
+                         ids=["one-full-wave", "queries-beyond-workspace", "split-tail"])
+def test_work_split_paths(lib, orc, H, T_c, T_q, launches):
+    """The attention's three layouts: whole 256-row blocks filling exactly one
+    wave (148 on a B200: no split, one kernel), more query rows than the
+    workspace holds partials for (no split), and a split tail merged by a
+    second kernel; each against the oracle."""
+    import torch
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148 and H == 37:
+        pytest.skip("the one-wave case assumes 148 SMs")
+    assert lib.attention_launches(2, T_c, H, T_q) == launches
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i in range(2):
+        K = synth.k_with_offsets_bf16(90 + i, T_c, H, (T_c, H, 128))
+        V = synth.gaussian_bf16(90 + i, T_c, H, synth.T_V, (T_c, H, 128))
+        b = lib.ChunkBuffer(T_c, H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), b, ws)
+        bufs.append(b)
+        qs.append(orc.quantize_chunk(K, V))
+    Q = synth.gaussian_bf16(95, T_c, H, synth.T_Q, (T_q, H, 128))
+    O = torch.empty((T_q, H, 128), dtype=torch.float32, device="cuda")
+    lib.attention(bufs, dev_bf16(Q), O, ws)
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    rows = sample_rows(T_q, n_random=16, seed=H)
+    ref = orc.attention_f64(qs, Q, rows=rows)
+    assert_attention_close(host_bf16_to_f64(O)[rows], ref, f"H={H} T_q={T_q}")
