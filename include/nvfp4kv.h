@@ -166,6 +166,48 @@ nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const void* V, int 
                                               int d, const nvfp4kv_chunk_view* out,
                                               nvfp4kv_stream_t stream);
 
+/* ------------------------------------------------------------------ sequence parallel */
+
+/*
+ * The chunk quantizer in three steps, for a chunk whose tokens are split over
+ * several GPUs (Ulysses-style sequence parallelism: the DeepRead page, Method
+ * > 推理基础设施, ships the 4-bit cache between GPUs instead of bf16).  Each
+ * GPU holds one contiguous shard of the chunk's tokens, [t0, t0 + T_local),
+ * for all H heads; every shard but the last starts and ends on a 64-token
+ * boundary, so that the K-smoothing segments of the one-GPU definition (the
+ * sequential sums over 64 tokens) fall inside one shard.  Composed as
+ *   stats (each shard) -> gather the segment statistics of all shards in
+ *   token order and the maximum of their max|V| -> finalize (every GPU, same
+ *   result) -> encode (each shard),
+ * the codes, scales, mean and tensor scales equal nvfp4kv_quantize_chunk's
+ * on the whole chunk bit for bit.
+ */
+
+/* Per shard: K's per-segment column sums psum [ceil(T_local/64)][H*d] (fp32,
+ * token order inside each segment), column minima / maxima pmin, pmax (same
+ * shape, bf16), and max |V| over the shard (*vmax, device float).  ws: a
+ * workspace of nvfp4kv_workspace_bytes(T_local, H, d). */
+nvfp4kv_status nvfp4kv_chunk_stats(const void* K, const void* V, int T_local, int H, int d,
+                                   float* psum, void* pmin, void* pmax, float* vmax, void* ws,
+                                   nvfp4kv_stream_t stream);
+
+/* From the statistics of all nseg = ceil(T/64) segments of the chunk (T tokens,
+ * shards concatenated in token order) and the chunk's max |V|: the mean
+ * k_mean [H][d] and tensor_scales {s_K, s_V}, exactly as the one-GPU
+ * quantizer forms them.  ws: a workspace of nvfp4kv_workspace_bytes(1, H, d)
+ * or larger. */
+nvfp4kv_status nvfp4kv_chunk_finalize(const float* psum, const void* pmin, const void* pmax,
+                                      int nseg, int T, int H, int d, const float* vmax,
+                                      float* k_mean, float* tensor_scales, void* ws,
+                                      nvfp4kv_stream_t stream);
+
+/* Per shard: codes and block scales of its T_local tokens (out's k/v codes and
+ * scales, laid out as a chunk of T_local tokens) with the chunk's k_mean and
+ * tensor_scales.  out->k_mean and out->tensor_scales are not used. */
+nvfp4kv_status nvfp4kv_chunk_encode(const void* K, const void* V, int T_local, int H, int d,
+                                    const float* k_mean, const float* tensor_scales,
+                                    const nvfp4kv_chunk_view* out, nvfp4kv_stream_t stream);
+
 /* ------------------------------------------------------------------ weights / activations */
 
 /* Block shape of nvfp4kv_quantize_matrix. */

@@ -70,6 +70,9 @@ def load():
         "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp]),
         "nvfp4kv_attention_launches": (i32, [i32, i32, i32, i32, i32]),
         "nvfp4kv_matrix_workspace_bytes": (sz, []),
+        "nvfp4kv_chunk_stats": (st, [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
+        "nvfp4kv_chunk_finalize": (st, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "nvfp4kv_chunk_encode": (st, [vp, vp, i32, i32, i32, vp, vp, cv, vp]),
         "nvfp4kv_quantize_matrix": (st, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
         "kvcache_pool_bytes": (sz, [cfgp]),
         "kvcache_create": (st, [cfgp, vp, vp, ctypes.POINTER(vp)]),
@@ -133,6 +136,44 @@ def version() -> str:
 
 def chunk_bytes(T_c, H, d=HEAD_DIM) -> int:
     return int(load().nvfp4kv_chunk_bytes(T_c, H, d))
+
+
+def chunk_stats(K, V, ws, stream=None):
+    """Per-shard statistics of the sequence-parallel quantizer: psum [nseg][H*d]
+    fp32, pmin / pmax [nseg][H*d] bf16, vmax [1] fp32."""
+    import torch
+    T, H, d = K.shape
+    nseg = (T + 63) // 64
+    psum = torch.empty((nseg, H * d), dtype=torch.float32, device=K.device)
+    pmin = torch.empty((nseg, H * d), dtype=torch.bfloat16, device=K.device)
+    pmax = torch.empty((nseg, H * d), dtype=torch.bfloat16, device=K.device)
+    vmax = torch.empty(1, dtype=torch.float32, device=K.device)
+    _check(load().nvfp4kv_chunk_stats(_ptr(K), _ptr(V), T, H, d, _ptr(psum), _ptr(pmin),
+                                      _ptr(pmax), _ptr(vmax), _ptr(ws), _stream(stream)),
+           "nvfp4kv_chunk_stats")
+    return psum, pmin, pmax, vmax
+
+
+def chunk_finalize(psum, pmin, pmax, vmax, T, H, ws, d=HEAD_DIM, stream=None):
+    """Mean [H][d] and tensor scales [2] of a chunk from all of its segments'
+    statistics (token order) and its max |V|."""
+    import torch
+    k_mean = torch.empty((H, d), dtype=torch.float32, device=psum.device)
+    scales = torch.empty(2, dtype=torch.float32, device=psum.device)
+    _check(load().nvfp4kv_chunk_finalize(_ptr(psum), _ptr(pmin), _ptr(pmax), psum.shape[0], T,
+                                         H, d, _ptr(vmax), _ptr(k_mean), _ptr(scales), _ptr(ws),
+                                         _stream(stream)),
+           "nvfp4kv_chunk_finalize")
+    return k_mean, scales
+
+
+def chunk_encode(K, V, k_mean, tensor_scales, out: "ChunkBuffer", stream=None):
+    """Codes and block scales of a token shard with the chunk's mean and scales."""
+    T, H, d = K.shape
+    _check(load().nvfp4kv_chunk_encode(_ptr(K), _ptr(V), T, H, d, _ptr(k_mean),
+                                       _ptr(tensor_scales), ctypes.byref(out.view),
+                                       _stream(stream)),
+           "nvfp4kv_chunk_encode")
 
 
 BLOCKS_1D, TILES_2D = 1, 2

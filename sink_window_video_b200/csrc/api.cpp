@@ -208,6 +208,48 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
     return launch_quantize(K, V, T_c, H, *out, ws, (cudaStream_t)stream);
 }
 
+nvfp4kv_status nvfp4kv_chunk_stats(const void* K, const void* V, int T_local, int H, int d,
+                                   float* psum, void* pmin, void* pmax, float* vmax, void* ws,
+                                   nvfp4kv_stream_t stream) {
+    if (!K || !V || !psum || !pmin || !pmax || !vmax || !ws || !valid_shape(T_local, H, d))
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(psum) || !aligned16(pmin) ||
+        !aligned16(pmax) || !aligned256(ws) || (reinterpret_cast<uintptr_t>(vmax) & 3u) != 0)
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_sp_stats(K, V, T_local, H, psum, pmin, pmax, vmax, ws, (cudaStream_t)stream);
+}
+
+nvfp4kv_status nvfp4kv_chunk_finalize(const float* psum, const void* pmin, const void* pmax,
+                                      int nseg, int T, int H, int d, const float* vmax,
+                                      float* k_mean, float* tensor_scales, void* ws,
+                                      nvfp4kv_stream_t stream) {
+    if (!psum || !pmin || !pmax || !vmax || !k_mean || !tensor_scales || !ws ||
+        !valid_shape(T, H, d) || nseg != (T + 63) / 64)
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned256(ws) || (reinterpret_cast<uintptr_t>(k_mean) & 15u) != 0)
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_sp_finalize(psum, pmin, pmax, nseg, T, H, vmax, k_mean, tensor_scales, ws,
+                              (cudaStream_t)stream);
+}
+
+nvfp4kv_status nvfp4kv_chunk_encode(const void* K, const void* V, int T_local, int H, int d,
+                                    const float* k_mean, const float* tensor_scales,
+                                    const nvfp4kv_chunk_view* out, nvfp4kv_stream_t stream) {
+    if (!K || !V || !k_mean || !tensor_scales || !out || !valid_shape(T_local, H, d) ||
+        !out->k_codes || !out->k_scales || !out->v_codes || !out->v_scales)
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(out->k_codes) || !aligned16(out->v_codes) ||
+        (reinterpret_cast<uintptr_t>(k_mean) & 15u) != 0)
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_sp_encode(K, V, T_local, H, k_mean, tensor_scales, *out, (cudaStream_t)stream);
+}
+
 size_t nvfp4kv_matrix_workspace_bytes(void) { return matrix_workspace_bytes(); }
 
 nvfp4kv_status nvfp4kv_quantize_matrix(const void* X, int M, int N, int mode, void* codes,

@@ -64,6 +64,17 @@ AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capac
 nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
                                const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream);
 
+// Sequence-parallel phases of the chunk quantizer (quant.cu).
+nvfp4kv_status launch_sp_stats(const void* K, const void* V, int T_local, int H, float* psum,
+                               void* pmin, void* pmax, float* vmax, void* ws,
+                               cudaStream_t stream);
+nvfp4kv_status launch_sp_finalize(const float* psum, const void* pmin, const void* pmax,
+                                  int nseg, int T, int H, const float* vmax, float* k_mean,
+                                  float* tensor_scales, void* ws, cudaStream_t stream);
+nvfp4kv_status launch_sp_encode(const void* K, const void* V, int T_local, int H,
+                                const float* k_mean, const float* tensor_scales,
+                                const nvfp4kv_chunk_view& out, cudaStream_t stream);
+
 // Weight / activation quantizer (matrix_quant.cu): workspace = control block +
 // per-CTA partial maxima.
 size_t matrix_workspace_bytes();

@@ -419,6 +419,79 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
     stamp(a, 7);
 }
 
+// ---------------------------------------------------------------- sequence-parallel phases
+//
+// The quantizer split at its global reductions, for a chunk whose tokens are
+// spread over several GPUs (one contiguous, 64-token-aligned shard each):
+//   stats:    per shard, the K column statistics of its 64-token segments and
+//             its max |V| (atomicMax on the float's bits: non-negative floats
+//             order like their bit patterns);
+//   (the caller gathers every shard's segment statistics in token order and
+//    takes the maximum of the max |V| values)
+//   finalize: the mean and max |K - mean| per column from all segments, in
+//             segment order -- the same fp32 sequence as the one-GPU kernel;
+//   scales:   the two tensor scales;
+//   encode:   per shard, the encoding of its tokens with the chunk's mean and
+//             tensor scales.
+// Each is an ordinary launch (no grid barrier); the results equal the one-GPU
+// quantization bit for bit.
+
+__global__ void __launch_bounds__(kQuantThreads, 1) sp_stats_kernel(QuantArgs a,
+                                                                      unsigned* vmax_bits) {
+    __shared__ QuantShared sh;
+    const uint64_t keep = policy_keep();
+    const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    const int nw = gridDim.x * kQuantWarps;
+    for (int u = wg; u < a.nseg * a.ngroups; u += nw) stats_unit(a, u, keep);
+    phase_vmax(a, sh, keep);                 // per-CTA max |V| into vpart[blockIdx.x] ...
+    if (threadIdx.x == 0) atomicMax(vmax_bits, __float_as_uint(a.vpart[blockIdx.x]));
+}
+
+__global__ void __launch_bounds__(kQuantThreads, 1) sp_finalize_kernel(QuantArgs a) {
+    __shared__ QuantShared sh;
+    phase_finalize(a, sh);                   // k_mean, per-CTA max |K - mean| in kpart
+}
+
+__global__ void sp_scales_kernel(const float* kpart, int n_part, const float* vmax,
+                                 float* tensor_scales) {
+    __shared__ float red[32];
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < n_part; i += blockDim.x) m = fmaxf(m, kpart[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float A = 0.0f;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) A = fmaxf(A, red[i]);
+        const float V = *vmax;
+        tensor_scales[0] = A > 0.0f ? __fdiv_rn(A, kTensorScaleDiv) : 1.0f;
+        tensor_scales[1] = V > 0.0f ? __fdiv_rn(V, kTensorScaleDiv) : 1.0f;
+    }
+}
+
+// blockIdx.y: 0 encodes V, 1 encodes K.
+__global__ void __launch_bounds__(kQuantThreads, 1) sp_encode_kernel(QuantArgs a) {
+    __shared__ QuantShared sh;
+    const bool isK = blockIdx.y == 1;
+    const float st = a.tensor_scales[isK ? 0 : 1];
+    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+        const float D = __fmul_rn(e4m3_to_f32((uint32_t)c), st);
+        sh.tab[c] = make_float2(D, D > 0.0f ? __frcp_rn(D) : 0.0f);
+    }
+    __syncthreads();
+    const EncodeConsts c = encode_consts(st);
+    const uint64_t release = policy_release();
+    const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    const int nw = gridDim.x * kQuantWarps;
+    const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
+    for (int u = wg; u < a.H * tiles; u += nw) {
+        const int h = u / tiles;
+        const int tile = u - h * tiles;
+        encode_unit(a, sh, isK, h, tile * kEncTokens, c.s, c.fast, c.ms6, c.ms4, c.rm, release);
+    }
+}
+
 // ---------------------------------------------------------------- dequantize
 
 // One thread per (head, token, 8-channel group): x = decode(q) * (decode(sb) * s)
@@ -570,6 +643,84 @@ nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,
     check_formats_kernel<<<blocks, threads, 0, stream>>>(
         op, static_cast<const float*>(in), static_cast<const uint8_t*>(in),
         static_cast<uint8_t*>(out), static_cast<float*>(out), n);
+    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+int sm_count_cached() {
+    static int sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (sms[dev] == 0 &&
+        cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms[dev] = 0;
+    return sms[dev];
+}
+
+nvfp4kv_status launch_sp_stats(const void* K, const void* V, int T_local, int H, float* psum,
+                               void* pmin, void* pmax, float* vmax, void* ws,
+                               cudaStream_t stream) {
+    const int G = sm_count_cached();
+    if (G <= 0) return NVFP4KV_ERR_CUDA;
+    const WsLayout L = ws_layout(T_local, H);
+    QuantArgs a = {};
+    a.K = static_cast<const uint4*>(K);
+    a.V = static_cast<const uint4*>(V);
+    a.T = T_local;
+    a.H = H;
+    a.HD = H * kHeadDim;
+    a.nseg = (T_local + kSegment - 1) / kSegment;
+    a.ngroups = (a.HD + 255) / 256;
+    a.psum = psum;
+    a.pmin = static_cast<uint32_t*>(pmin);
+    a.pmax = static_cast<uint32_t*>(pmax);
+    a.vpart = reinterpret_cast<float*>(static_cast<char*>(ws) + L.vpart);
+    a.one = 1.0f;
+    if (cudaMemsetAsync(vmax, 0, sizeof(float), stream) != cudaSuccess) return NVFP4KV_ERR_CUDA;
+    sp_stats_kernel<<<G, kQuantThreads, 0, stream>>>(a, reinterpret_cast<unsigned*>(vmax));
+    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+nvfp4kv_status launch_sp_finalize(const float* psum, const void* pmin, const void* pmax,
+                                  int nseg, int T, int H, const float* vmax, float* k_mean,
+                                  float* tensor_scales, void* ws, cudaStream_t stream) {
+    const int HD = H * kHeadDim;
+    const int nblocks = HD / kFinCols;
+    const int G = min(nblocks, kMaxGrid);
+    QuantArgs a = {};
+    a.T = T;
+    a.H = H;
+    a.HD = HD;
+    a.nseg = nseg;
+    a.psum = const_cast<float*>(psum);
+    a.pmin = static_cast<uint32_t*>(const_cast<void*>(pmin));
+    a.pmax = static_cast<uint32_t*>(const_cast<void*>(pmax));
+    a.k_mean = k_mean;
+    a.kpart = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_layout(1, H).kpart);
+    sp_finalize_kernel<<<G, kQuantThreads, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
+    sp_scales_kernel<<<1, 1024, 0, stream>>>(a.kpart, G, vmax, tensor_scales);
+    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+nvfp4kv_status launch_sp_encode(const void* K, const void* V, int T_local, int H,
+                                const float* k_mean, const float* tensor_scales,
+                                const nvfp4kv_chunk_view& out, cudaStream_t stream) {
+    const int G = sm_count_cached();
+    if (G <= 0) return NVFP4KV_ERR_CUDA;
+    QuantArgs a = {};
+    a.K = static_cast<const uint4*>(K);
+    a.V = static_cast<const uint4*>(V);
+    a.T = T_local;
+    a.H = H;
+    a.HD = H * kHeadDim;
+    a.k_codes = out.k_codes;
+    a.k_scales = out.k_scales;
+    a.v_codes = out.v_codes;
+    a.v_scales = out.v_scales;
+    a.k_mean = const_cast<float*>(k_mean);
+    a.tensor_scales = const_cast<float*>(tensor_scales);
+    a.one = 1.0f;
+    sp_encode_kernel<<<dim3((G + 1) / 2, 2), kQuantThreads, 0, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 

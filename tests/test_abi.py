@@ -84,6 +84,14 @@ def test_rejects_bad_arguments_without_device_work(L):
     assert m(FAKE, 24, 32, 2, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_UNSUPPORTED
     assert m(FAKE + 8, 16, 32, 2, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_ALIGNMENT
     assert L.nvfp4kv_matrix_workspace_bytes() >= 256
+    assert L.nvfp4kv_chunk_stats(None, FAKE, 64, 2, 128, FAKE, FAKE, FAKE, FAKE, FAKE, None) \
+        == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_chunk_stats(FAKE, FAKE, 64, 2, 96, FAKE, FAKE, FAKE, FAKE, FAKE, None) \
+        == swv.ERR_UNSUPPORTED
+    assert L.nvfp4kv_chunk_finalize(FAKE, FAKE, FAKE, 3, 200, 2, 128, FAKE, FAKE, FAKE, FAKE,
+                                    None) == swv.ERR_INVALID_ARG           # 200 tokens: 4 segments
+    assert L.nvfp4kv_chunk_encode(FAKE, FAKE, 64, 2, 128, FAKE, FAKE, None, None) \
+        == swv.ERR_INVALID_ARG
     assert L.nvfp4kv_workspace_init(None, 256, None) == swv.ERR_INVALID_ARG
 
 
