@@ -56,7 +56,7 @@ NCU_TRAFFIC = {
     "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
                   "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
-                 "8c313008b89b811449016aa51c0c8d49d2a1c6a635c3f210927caccf8c5620b2", 97300224),
+                 "e1ad8f385bece23e3d0be852eaa7b32c867a427aa21558911cf0f7994c3de6f1", 95927808),
 }
 
 
