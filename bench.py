@@ -317,14 +317,48 @@ def run_ours(args, rank, world, local):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
 
     matrix = run_matrix_quant(swv, pool, stream) if not args.no_matrix else None
+    dequant = run_dequant(swv, cache, stream) if not args.no_matrix else None
 
     rollouts = None
     if not args.no_rollout:
         rollouts = [run_rollout(swv, cfg, pool, O, stream, world) for cfg in ROLLOUTS]
 
     return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
-                e2e_ms=e2e_ms, rollouts=rollouts, matrix=matrix,
+                e2e_ms=e2e_ms, rollouts=rollouts, matrix=matrix, dequant=dequant,
                 attn_launches=swv.attention_launches(len(cache.keyset(0)), T, H, T))
+
+
+# ------------------------------------------------------------------ standalone de-quantization
+
+def run_dequant(swv, cache, stream, launches=40):
+    """nvfp4kv_dequantize of K and V of the cache's chunks to bf16 (rotating over
+    the 5 chunks of the key set): reads codes, scales, mean and tensor scales,
+    writes 2 x [7040, 24, 128] bf16."""
+    import torch
+    peaks, src = load_peaks()
+    hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    T, H, d = CFG["T_c"], CFG["H"], CFG["d"]
+    chunks = [cache.chunk(0, n) for n in cache.keyset(0)]
+    Ko = torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda")
+    Vo = torch.empty_like(Ko)
+    for i in range(3):
+        swv.dequantize(chunks[i % len(chunks)], Ko, Vo)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(launches)]
+    torch.cuda.synchronize()
+    for i, (e0, e1) in enumerate(ev):
+        e0.record(stream)
+        swv.dequantize(chunks[i % len(chunks)], Ko, Vo)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * sum(e0.elapsed_time(e1) for e0, e1 in ev) / launches
+    n = T * H * d
+    nbytes = 2 * (n // 2 + n // 16) + H * d * 4 + 8 + 2 * 2 * n
+    gbs = nbytes / (us / 1e6) / 1e9
+    return {"kernel": "nvfp4kv_dequantize (K and V to bf16)", "us_per_launch": us,
+            "bytes_per_launch": nbytes, "achieved": gbs, "unit": "GB/s", "peak": hpeak,
+            "frac": gbs / hpeak, "bound": "hbm", "gpu_launches_per_call": 1,
+            "peak_source": f"{src} hbm"}
 
 
 # ------------------------------------------------------------------ weights / activations
@@ -579,6 +613,8 @@ def main():
             line["rollouts"] = r["rollouts"]
         if r["matrix"] is not None:
             line["matrix_quantize"] = r["matrix"]
+        if r["dequant"] is not None:
+            line["dequantize"] = r["dequant"]
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = OracleSample(rows=args.ref_rows).baseline()
         print(json.dumps(line))

@@ -119,6 +119,17 @@ def _dtype_code(t):
     raise TypeError(f"output dtype {t.dtype} is not float32 or bfloat16")
 
 
+def _check_qo(Q, O, H, d):
+    """Q: contiguous bf16 [T_q, H, d]; O: contiguous, same element count."""
+    import torch
+    if Q.dtype != torch.bfloat16 or Q.dim() != 3 or tuple(Q.shape[1:]) != (H, d) \
+            or not Q.is_contiguous():
+        raise ValueError(f"Q must be a contiguous bf16 [T_q, {H}, {d}] tensor, "
+                         f"got {Q.dtype} {tuple(Q.shape)}")
+    if not O.is_contiguous() or O.numel() != Q.numel():
+        raise ValueError(f"O of shape {tuple(O.shape)} does not match Q {tuple(Q.shape)}")
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -297,9 +308,18 @@ def quantize_chunk(K, V, out: ChunkBuffer, ws, stream=None):
 
 
 def dequantize(chunk: ChunkBuffer, K_out=None, V_out=None, stream=None):
-    """Write de-quantized [T_c, H, d] K and/or V (float32 or bf16 tensors)."""
-    t = K_out if K_out is not None else V_out
-    dtype = _dtype_code(t)
+    """Write de-quantized [T_c, H, d] K and/or V: contiguous tensors of one
+    dtype (float32 or bf16), the dtype the library writes both in."""
+    outs = [t for t in (K_out, V_out) if t is not None]
+    if not outs:
+        return
+    dtype = _dtype_code(outs[0])
+    for t in outs:
+        if _dtype_code(t) != dtype:
+            raise TypeError("K_out and V_out must have the same dtype")
+        if not t.is_contiguous() or t.numel() != chunk.T_c * chunk.H * chunk.d:
+            raise ValueError(f"output of shape {tuple(t.shape)} is not a contiguous "
+                             f"[{chunk.T_c}, {chunk.H}, {chunk.d}] tensor")
     _check(load().nvfp4kv_dequantize(ctypes.byref(chunk.view), chunk.T_c, chunk.H, chunk.d,
                                      _ptr(K_out), _ptr(V_out), dtype, _stream(stream)),
            "nvfp4kv_dequantize")
@@ -312,6 +332,7 @@ def attention(chunks, Q, O, ws, softmax_scale=0.0, stream=None):
     first = chunks[0] if chunks else None
     T_c = first.T_c if hasattr(first, "T_c") else 0
     T_q, H, d = Q.shape
+    _check_qo(Q, O, H, d)
     _check(load().nvfp4kv_attention(arr, len(views), T_c, H, d, _ptr(Q), T_q, _ptr(O),
                                     _dtype_code(O), float(softmax_scale), _ptr(ws),
                                     _stream(stream)),
@@ -392,6 +413,7 @@ class KVCache:
 
     def attention(self, layer, Q, O, softmax_scale=0.0, stream=None):
         T_q = Q.shape[0]
+        _check_qo(Q, O, self.H, self.d)
         _check(load().sink_window_attention(self._h, layer, _ptr(Q), T_q, _ptr(O),
                                             _dtype_code(O), float(softmax_scale),
                                             _stream(stream)),

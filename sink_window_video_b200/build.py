@@ -23,6 +23,7 @@ COMMON = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
 PER_FILE = {
     "quant.cu": ["-fmad=false"],
     "matrix_quant.cu": ["-fmad=false"],
+    "dequant.cu": ["-fmad=false"],
 }
 
 

@@ -82,6 +82,7 @@ nvfp4kv_status launch_quantize_matrix(const void* X, int M, int N, int mode, voi
                                       void* scales, float* tensor_scale, void* ws,
                                       cudaStream_t stream);
 
+int sm_count_cached();
 nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, void* K_out,
                                  void* V_out, int out_dtype, cudaStream_t stream);
 

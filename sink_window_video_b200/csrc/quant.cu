@@ -1,5 +1,5 @@
 // quant.cu -- chunk-level NVFP4 quantization of K and V with K-smoothing and
-// Four-Over-Six block scales, its inverse, and the format-check kernel.
+// Four-Over-Six block scales, and the format-check kernel.
 //
 // Method ("2605-LongLive2" DeepRead page, Method > 推理基础设施 and
 // 训练基础设施; tailorednewshub page, Inferenza W4A4 NVFP4): per chunk and per
@@ -492,52 +492,6 @@ __global__ void __launch_bounds__(kQuantThreads, 1) sp_encode_kernel(QuantArgs a
     }
 }
 
-// ---------------------------------------------------------------- dequantize
-
-// One thread per (head, token, 8-channel group): x = decode(q) * (decode(sb) * s)
-// (+ mean for K); output [T][H][d] fp32 or bf16 (nearest even).
-__global__ void dequant_kernel(const uint8_t* codes, const uint8_t* scales, const float* mean,
-                               const float* tensor_scales, int which, int T, int H, void* out,
-                               int out_bf16) {
-    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t total = (size_t)H * T * 16;
-    if (idx >= total) return;
-    const int g = (int)(idx & 15);
-    const size_t row = idx >> 4;                   // h * T + t
-    const int h = (int)(row / T);
-    const int t = (int)(row - (size_t)h * T);
-    const float s = tensor_scales[which];
-    const uint32_t q = reinterpret_cast<const uint32_t*>(codes)[row * 16 + g];
-    const float D = __fmul_rn(e4m3_to_f32(scales[row * 8 + (g >> 1)]), s);
-    uint32_t hq[4];
-    cvt_e2m1x8_to_f16x2(q, hq);
-    float x[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        x[2 * j] = __fmul_rn(f16lo(hq[j]), D);
-        x[2 * j + 1] = __fmul_rn(f16hi(hq[j]), D);
-    }
-    if (mean) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = __fadd_rn(x[i], mean[h * kHeadDim + g * 8 + i]);
-    }
-    const size_t o = ((size_t)t * H + h) * kHeadDim + g * 8;
-    if (out_bf16) {
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            __nv_bfloat162 p = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
-            w[j] = *reinterpret_cast<uint32_t*>(&p);
-        }
-        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + o) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-        float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + o);
-        p[0] = make_float4(x[0], x[1], x[2], x[3]);
-        p[1] = make_float4(x[4], x[5], x[6], x[7]);
-    }
-}
-
 // ---------------------------------------------------------------- format checks
 
 __global__ void check_formats_kernel(int op, const float* fin, const uint8_t* bin, uint8_t* bout,
@@ -617,22 +571,6 @@ nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
                                                 dim3(g_quant_grid[dev]), dim3(kQuantThreads),
                                                 args, 0, stream);
     return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
-}
-
-nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, void* K_out,
-                                 void* V_out, int out_dtype, cudaStream_t stream) {
-    const size_t total = (size_t)H * T * 16;
-    const int threads = 256;
-    const unsigned blocks = (unsigned)((total + threads - 1) / threads);
-    if (K_out)
-        dequant_kernel<<<blocks, threads, 0, stream>>>(in.k_codes, in.k_scales, in.k_mean,
-                                                       in.tensor_scales, 0, T, H, K_out,
-                                                       out_dtype);
-    if (V_out)
-        dequant_kernel<<<blocks, threads, 0, stream>>>(in.v_codes, in.v_scales, nullptr,
-                                                       in.tensor_scales, 1, T, H, V_out,
-                                                       out_dtype);
-    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
 nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,

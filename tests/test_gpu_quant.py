@@ -138,14 +138,64 @@ def test_dequantize_bit_exact(lib, orc, bf16_out):
     assert np.array_equal(Kg, Kr) and np.array_equal(Vg, Vr)
 
 
-def test_dequantize_full_size_bit_exact(lib, orc):
+@pytest.mark.parametrize("T,H", [(1, 1), (13, 3), (200, 5), (37, 33), (64, 40), (9, 70)])
+@pytest.mark.parametrize("bf16_out", [False, True])
+def test_dequantize_ragged_tiles_bit_exact(lib, orc, T, H, bf16_out):
+    """Token counts that leave a partial tile, head counts below a tile's
+    width, across two and three head blocks."""
+    import torch
+    K = synth.k_with_offsets_bf16(57, T, H, (T, H, 128), outlier_mult=20.0)
+    V = synth.gaussian_bf16(57, T, H, synth.T_V, (T, H, 128))
+    out, _ = _gpu_quant(lib, K, V)
+    q = orc.quantize_chunk(K, V)
+    _assert_same(out.to_host(), q, f"T={T} H={H}")
+    dt = torch.bfloat16 if bf16_out else torch.float32
+    Kd = torch.empty((T, H, 128), dtype=dt, device="cuda")
+    Vd = torch.empty((T, H, 128), dtype=dt, device="cuda")
+    lib.dequantize(out, Kd, Vd)
+    torch.cuda.synchronize()
+    Kr = orc.dequantize_tensor(q["k_codes"], q["k_scales"], q["k_mean"], q["s_k"], T, H, 128)
+    Vr = orc.dequantize_tensor(q["v_codes"], q["v_scales"], None, q["s_v"], T, H, 128)
+    for name, got, want in (("K", Kd, Kr), ("V", Vd, Vr)):
+        if bf16_out:
+            g = got.view(torch.int16).cpu().numpy().view(np.uint16)
+            w = orc.f32_to_bf16(want)
+        else:
+            g, w = got.cpu().numpy().view(np.uint32), want.view(np.uint32)
+        assert np.array_equal(g, w), f"{name} T={T} H={H}"
+
+
+def test_dequantize_rejects_mixed_or_short_outputs(lib):
+    import torch
+    K, V, _ = synth.tiny_chunk(1)
+    T, H, d = K.shape
+    out, _ = _gpu_quant(lib, K, V)
+    Kd = torch.empty((T, H, d), dtype=torch.float32, device="cuda")
+    with pytest.raises(TypeError):
+        lib.dequantize(out, Kd, torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        lib.dequantize(out, Kd, torch.empty((T - 1, H, d), dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("which", ["K", "V"])
+def test_dequantize_full_size_bit_exact(lib, orc, which):
+    """One tensor at a time (the other output pointer NULL), full chunk size;
+    K to fp32, V to bf16."""
     import torch
     K, V = synth.quant_chunk(2)
     T, H, d = K.shape
     out, _ = _gpu_quant(lib, K, V)
-    Kd = torch.empty((T, H, d), dtype=torch.float32, device="cuda")
-    lib.dequantize(out, K_out=Kd)
-    torch.cuda.synchronize()
     q = orc.quantize_chunk(K, V)
-    Kr = orc.dequantize_tensor(q["k_codes"], q["k_scales"], q["k_mean"], q["s_k"], T, H, d)
-    assert np.array_equal(Kd.cpu().numpy().view(np.uint32), Kr.view(np.uint32))
+    if which == "K":
+        Kd = torch.empty((T, H, d), dtype=torch.float32, device="cuda")
+        lib.dequantize(out, K_out=Kd)
+        torch.cuda.synchronize()
+        Kr = orc.dequantize_tensor(q["k_codes"], q["k_scales"], q["k_mean"], q["s_k"], T, H, d)
+        assert np.array_equal(Kd.cpu().numpy().view(np.uint32), Kr.view(np.uint32))
+    else:
+        Vd = torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda")
+        lib.dequantize(out, V_out=Vd)
+        torch.cuda.synchronize()
+        Vr = orc.dequantize_tensor(q["v_codes"], q["v_scales"], None, q["s_v"], T, H, d)
+        Vg = Vd.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(Vg, orc.f32_to_bf16(Vr))
