@@ -56,7 +56,9 @@ NCU_TRAFFIC = {
     "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
                   "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
-                 "e1ad8f385bece23e3d0be852eaa7b32c867a427aa21558911cf0f7994c3de6f1", 95927808),
+                 "6a8cb7ce1a56316e2dad4dd9c3ecd74d349d1a1ea48f29dcccb9dfda8cd02dec", 97600000),
+    "dequantize": ("sink_window_video_b200/csrc/dequant.cu",
+                   "abbdbf999d98f485296aa8637dda0439dda52de694237ef5f4cb6239b7ebf0f9", 51689728),
 }
 
 
@@ -358,7 +360,7 @@ def run_dequant(swv, cache, stream, launches=40):
     return {"kernel": "nvfp4kv_dequantize (K and V to bf16)", "us_per_launch": us,
             "bytes_per_launch": nbytes, "achieved": gbs, "unit": "GB/s", "peak": hpeak,
             "frac": gbs / hpeak, "bound": "hbm", "gpu_launches_per_call": 1,
-            "peak_source": f"{src} hbm"}
+            "traffic": ncu_traffic("dequantize"), "peak_source": f"{src} hbm"}
 
 
 # ------------------------------------------------------------------ weights / activations

@@ -208,6 +208,36 @@ nvfp4kv_status nvfp4kv_chunk_encode(const void* K, const void* V, int T_local, i
                                     const float* k_mean, const float* tensor_scales,
                                     const nvfp4kv_chunk_view* out, nvfp4kv_stream_t stream);
 
+/* ------------------------------------------------------------------ head parallel */
+
+/*
+ * The chunk quantizer for a chunk whose heads are split over several GPUs:
+ * each GPU holds all T tokens of its heads [h0, h1) as a [T, h1 - h0, d]
+ * tensor.  The K mean and the blocks are per head; only the two tensor scales
+ * couple the heads (one FP32 scale per chunk and tensor, the DeepRead page,
+ * Method > 推理基础设施), and s = amax / 2688 needs the amax of the whole
+ * tensor.  Composed as
+ *   nvfp4kv_chunk_stats (own heads) -> nvfp4kv_chunk_amax (own heads: k_mean
+ *   and the two amaxes) -> the maximum of each amax over the GPUs (one
+ *   all-reduce of two floats) -> nvfp4kv_tensor_scales_from_amax ->
+ *   nvfp4kv_chunk_encode (own heads),
+ * each GPU's codes, scales and mean equal those heads of
+ * nvfp4kv_quantize_chunk's result on the whole chunk, and every GPU's tensor
+ * scales equal the whole chunk's, bit for bit.
+ */
+
+/* nvfp4kv_chunk_finalize's inputs and k_mean; instead of the tensor scales,
+ * amax[0] = max |RN(K - mean)| and amax[1] = *vmax (device floats). */
+nvfp4kv_status nvfp4kv_chunk_amax(const float* psum, const void* pmin, const void* pmax,
+                                  int nseg, int T, int H, int d, const float* vmax,
+                                  float* k_mean, float* amax, void* ws,
+                                  nvfp4kv_stream_t stream);
+
+/* tensor_scales[i] = amax[i] / 2688 (fp32, correctly rounded), or 1 where
+ * amax[i] is 0; both device arrays of 2 floats. */
+nvfp4kv_status nvfp4kv_tensor_scales_from_amax(const float* amax, float* tensor_scales,
+                                               nvfp4kv_stream_t stream);
+
 /* ------------------------------------------------------------------ weights / activations */
 
 /* Block shape of nvfp4kv_quantize_matrix. */

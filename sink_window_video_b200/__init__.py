@@ -72,6 +72,8 @@ def load():
         "nvfp4kv_matrix_workspace_bytes": (sz, []),
         "nvfp4kv_chunk_stats": (st, [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
         "nvfp4kv_chunk_finalize": (st, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "nvfp4kv_chunk_amax": (st, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "nvfp4kv_tensor_scales_from_amax": (st, [vp, vp, vp]),
         "nvfp4kv_chunk_encode": (st, [vp, vp, i32, i32, i32, vp, vp, cv, vp]),
         "nvfp4kv_quantize_matrix": (st, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
         "kvcache_pool_bytes": (sz, [cfgp]),
@@ -176,6 +178,31 @@ def chunk_finalize(psum, pmin, pmax, vmax, T, H, ws, d=HEAD_DIM, stream=None):
                                          _stream(stream)),
            "nvfp4kv_chunk_finalize")
     return k_mean, scales
+
+
+def chunk_amax(psum, pmin, pmax, vmax, T, H, ws, d=HEAD_DIM, k_mean=None, stream=None):
+    """Mean [H][d] (into k_mean when given) and the two amaxes [max |K - mean|,
+    max |V|] of a chunk, or of a head shard of it, from its segments'
+    statistics and its max |V|."""
+    import torch
+    if k_mean is None:
+        k_mean = torch.empty((H, d), dtype=torch.float32, device=psum.device)
+    amax = torch.empty(2, dtype=torch.float32, device=psum.device)
+    _check(load().nvfp4kv_chunk_amax(_ptr(psum), _ptr(pmin), _ptr(pmax), psum.shape[0], T, H, d,
+                                     _ptr(vmax), _ptr(k_mean), _ptr(amax), _ptr(ws),
+                                     _stream(stream)),
+           "nvfp4kv_chunk_amax")
+    return k_mean, amax
+
+
+def tensor_scales_from_amax(amax, out=None, stream=None):
+    """[s_K, s_V] = amax / 2688 (1 for a zero amax), on the device."""
+    import torch
+    if out is None:
+        out = torch.empty(2, dtype=torch.float32, device=amax.device)
+    _check(load().nvfp4kv_tensor_scales_from_amax(_ptr(amax), _ptr(out), _stream(stream)),
+           "nvfp4kv_tensor_scales_from_amax")
+    return out
 
 
 def chunk_encode(K, V, k_mean, tensor_scales, out: "ChunkBuffer", stream=None):

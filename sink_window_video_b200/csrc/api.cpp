@@ -232,8 +232,30 @@ nvfp4kv_status nvfp4kv_chunk_finalize(const float* psum, const void* pmin, const
     if (!aligned256(ws) || (reinterpret_cast<uintptr_t>(k_mean) & 15u) != 0)
         return NVFP4KV_ERR_ALIGNMENT;
     if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
-    return launch_sp_finalize(psum, pmin, pmax, nseg, T, H, vmax, k_mean, tensor_scales, ws,
+    return launch_sp_finalize(psum, pmin, pmax, nseg, T, H, vmax, k_mean, nullptr,
+                              tensor_scales, ws, (cudaStream_t)stream);
+}
+
+nvfp4kv_status nvfp4kv_chunk_amax(const float* psum, const void* pmin, const void* pmax,
+                                  int nseg, int T, int H, int d, const float* vmax,
+                                  float* k_mean, float* amax, void* ws,
+                                  nvfp4kv_stream_t stream) {
+    if (!psum || !pmin || !pmax || !vmax || !k_mean || !amax || !ws || !valid_shape(T, H, d) ||
+        nseg != (T + 63) / 64)
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned256(ws) || (reinterpret_cast<uintptr_t>(k_mean) & 15u) != 0)
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_sp_finalize(psum, pmin, pmax, nseg, T, H, vmax, k_mean, amax, nullptr, ws,
                               (cudaStream_t)stream);
+}
+
+nvfp4kv_status nvfp4kv_tensor_scales_from_amax(const float* amax, float* tensor_scales,
+                                               nvfp4kv_stream_t stream) {
+    if (!amax || !tensor_scales) return NVFP4KV_ERR_INVALID_ARG;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_scales_from_amax(amax, tensor_scales, (cudaStream_t)stream);
 }
 
 nvfp4kv_status nvfp4kv_chunk_encode(const void* K, const void* V, int T_local, int H, int d,

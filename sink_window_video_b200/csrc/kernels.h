@@ -70,7 +70,10 @@ nvfp4kv_status launch_sp_stats(const void* K, const void* V, int T_local, int H,
                                cudaStream_t stream);
 nvfp4kv_status launch_sp_finalize(const float* psum, const void* pmin, const void* pmax,
                                   int nseg, int T, int H, const float* vmax, float* k_mean,
-                                  float* tensor_scales, void* ws, cudaStream_t stream);
+                                  float* amax, float* tensor_scales, void* ws,
+                                  cudaStream_t stream);
+nvfp4kv_status launch_scales_from_amax(const float* amax, float* tensor_scales,
+                                       cudaStream_t stream);
 nvfp4kv_status launch_sp_encode(const void* K, const void* V, int T_local, int H,
                                 const float* k_mean, const float* tensor_scales,
                                 const nvfp4kv_chunk_view& out, cudaStream_t stream);

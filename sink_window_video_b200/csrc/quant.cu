@@ -452,8 +452,11 @@ __global__ void __launch_bounds__(kQuantThreads, 1) sp_finalize_kernel(QuantArgs
     phase_finalize(a, sh);                   // k_mean, per-CTA max |K - mean| in kpart
 }
 
+// max over the per-CTA partial maxima of |K - mean| and the given max |V|:
+// the two amaxes (amax_out, when given) and the tensor scales s = amax / 2688
+// (1 for an all-zero tensor; tensor_scales, when given).
 __global__ void sp_scales_kernel(const float* kpart, int n_part, const float* vmax,
-                                 float* tensor_scales) {
+                                 float* amax_out, float* tensor_scales) {
     __shared__ float red[32];
     float m = 0.0f;
     for (int i = threadIdx.x; i < n_part; i += blockDim.x) m = fmaxf(m, kpart[i]);
@@ -465,8 +468,14 @@ __global__ void sp_scales_kernel(const float* kpart, int n_part, const float* vm
         float A = 0.0f;
         for (int i = 0; i < (int)(blockDim.x >> 5); ++i) A = fmaxf(A, red[i]);
         const float V = *vmax;
-        tensor_scales[0] = A > 0.0f ? __fdiv_rn(A, kTensorScaleDiv) : 1.0f;
-        tensor_scales[1] = V > 0.0f ? __fdiv_rn(V, kTensorScaleDiv) : 1.0f;
+        if (amax_out) {
+            amax_out[0] = A;
+            amax_out[1] = V;
+        }
+        if (tensor_scales) {
+            tensor_scales[0] = A > 0.0f ? __fdiv_rn(A, kTensorScaleDiv) : 1.0f;
+            tensor_scales[1] = V > 0.0f ? __fdiv_rn(V, kTensorScaleDiv) : 1.0f;
+        }
     }
 }
 
@@ -620,7 +629,8 @@ nvfp4kv_status launch_sp_stats(const void* K, const void* V, int T_local, int H,
 
 nvfp4kv_status launch_sp_finalize(const float* psum, const void* pmin, const void* pmax,
                                   int nseg, int T, int H, const float* vmax, float* k_mean,
-                                  float* tensor_scales, void* ws, cudaStream_t stream) {
+                                  float* amax, float* tensor_scales, void* ws,
+                                  cudaStream_t stream) {
     const int HD = H * kHeadDim;
     const int nblocks = HD / kFinCols;
     const int G = min(nblocks, kMaxGrid);
@@ -636,7 +646,13 @@ nvfp4kv_status launch_sp_finalize(const float* psum, const void* pmin, const voi
     a.kpart = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_layout(1, H).kpart);
     sp_finalize_kernel<<<G, kQuantThreads, 0, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
-    sp_scales_kernel<<<1, 1024, 0, stream>>>(a.kpart, G, vmax, tensor_scales);
+    sp_scales_kernel<<<1, 1024, 0, stream>>>(a.kpart, G, vmax, amax, tensor_scales);
+    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+nvfp4kv_status launch_scales_from_amax(const float* amax, float* tensor_scales,
+                                       cudaStream_t stream) {
+    sp_scales_kernel<<<1, 32, 0, stream>>>(amax, 1, amax + 1, nullptr, tensor_scales);
     return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 

@@ -24,6 +24,12 @@ Shards: whole 64-token segments split as evenly as possible (shard_bounds), so
 that every K-smoothing segment lies in one shard.  H must divide by P.  The
 collectives are torch.distributed's (NCCL between GPUs); the layout steps
 between them are plain tensor reshapes.
+
+Head parallelism (quantize_chunk_heads): each rank already holds every token
+of its heads [h0, h1) (head_bounds).  The mean and the blocks are per head, so
+the one exchange per chunk is an all-reduce(max) of the two amaxes that set
+the tensor scales (reduce_amax); attention then runs on each rank's heads with
+no exchange at all.
 """
 import torch
 import torch.distributed as dist
@@ -154,6 +160,28 @@ def quantize_chunk_sp(K_local, V_local, T: int, ws, group=None):
         getattr(out, name).copy_(x)
     out.k_mean.copy_(k_mean[rank * Hp:(rank + 1) * Hp])
     out.tensor_scales.copy_(scales)
+    return out
+
+
+def reduce_amax(amax, group=None):
+    """The chunk's [max |K - mean|, max |V|] from every rank's: all-reduce(max)
+    of two floats, in place."""
+    dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    return amax
+
+
+def quantize_chunk_heads(K_heads, V_heads, ws, group=None):
+    """This rank's heads of the quantized chunk (a ChunkBuffer of all T tokens
+    and the rank's heads) from K, V [T, h1 - h0, d] of those heads; bit-equal
+    to those heads of the one-GPU quantization, with the whole chunk's tensor
+    scales."""
+    T, Hr, d = K_heads.shape
+    psum, pmin, pmax, vmax = lib.chunk_stats(K_heads, V_heads, ws)
+    out = lib.ChunkBuffer(T, Hr, d)
+    _, amax = lib.chunk_amax(psum, pmin, pmax, vmax, T, Hr, ws, k_mean=out.k_mean)
+    reduce_amax(amax, group)
+    lib.tensor_scales_from_amax(amax, out.tensor_scales)
+    lib.chunk_encode(K_heads, V_heads, out.k_mean, out.tensor_scales, out)
     return out
 
 

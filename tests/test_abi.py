@@ -92,6 +92,16 @@ def test_rejects_bad_arguments_without_device_work(L):
                                     None) == swv.ERR_INVALID_ARG           # 200 tokens: 4 segments
     assert L.nvfp4kv_chunk_encode(FAKE, FAKE, 64, 2, 128, FAKE, FAKE, None, None) \
         == swv.ERR_INVALID_ARG
+    a = L.nvfp4kv_chunk_amax
+    assert a(FAKE, FAKE, FAKE, 3, 200, 2, 128, FAKE, FAKE, FAKE, FAKE, None) \
+        == swv.ERR_INVALID_ARG                                            # 200 tokens: 4 segments
+    assert a(FAKE, FAKE, FAKE, 4, 200, 2, 128, FAKE, FAKE, None, FAKE, None) \
+        == swv.ERR_INVALID_ARG                                            # no amax output
+    assert a(FAKE, FAKE, FAKE, 4, 200, 2, 96, FAKE, FAKE, FAKE, FAKE, None) == swv.ERR_UNSUPPORTED
+    assert a(FAKE, FAKE, FAKE, 4, 200, 2, 128, FAKE, FAKE, FAKE, FAKE + 16, None) \
+        == swv.ERR_ALIGNMENT                                              # workspace not 256-aligned
+    assert L.nvfp4kv_tensor_scales_from_amax(None, FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_tensor_scales_from_amax(FAKE, None, None) == swv.ERR_INVALID_ARG
     assert L.nvfp4kv_workspace_init(None, 256, None) == swv.ERR_INVALID_ARG
 
 

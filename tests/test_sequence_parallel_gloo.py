@@ -3,8 +3,10 @@ sequence_parallel.py) with real collectives: 2 and 3 gloo ranks on CPU.  The
 data are the oracle's: the full chunk quantized in one piece, cut into token
 shards as each rank's encoder would produce them.  Checked: the gathered
 segment statistics equal those of the whole chunk (token order), every rank's
-head shard equals those heads of the one-piece quantization byte for byte, and
-queries and outputs round-trip between token and head shards."""
+head shard equals those heads of the one-piece quantization byte for byte,
+queries and outputs round-trip between token and head shards, and (head
+parallelism) the all-reduced amaxes of the ranks' own heads are the whole
+chunk's, whose quotients by 2688 are its tensor scales."""
 import os
 import socket
 
@@ -71,6 +73,19 @@ def _rank(rank, P, port, out):
         Qh = sp.exchange_queries(Qt[t0:t1].contiguous(), T)
         res["q"] = torch.equal(Qh, Qt[:, h0:h1])
         res["o"] = torch.equal(sp.exchange_outputs(Qh, T, H), Qt[t0:t1])
+        # head parallelism: this rank's heads alone -> its amaxes -> reduce_amax
+        # gives the whole chunk's, and amax / 2688 its tensor scales
+        qh = oracle.quantize_chunk(np.ascontiguousarray(K[:, h0:h1]), np.ascontiguousarray(V[:, h0:h1]))
+        kf, vf = synth.bf16_bits_to_f32(K), synth.bf16_bits_to_f32(V)
+        X = (kf[:, h0:h1] - qh["k_mean"][None]).astype(np.float32)
+        amax = torch.tensor([np.abs(X).max(), np.abs(vf[:, h0:h1]).max()], dtype=torch.float32)
+        sp.reduce_amax(amax)
+        Xf = (kf - q["k_mean"][None]).astype(np.float32)
+        res["amax"] = (np.array_equal(qh["k_mean"], q["k_mean"][h0:h1])
+                       and float(amax[0]) == float(np.abs(Xf).max())
+                       and float(amax[1]) == float(np.abs(vf).max())
+                       and np.float32(amax[0].item()) / np.float32(2688) == np.float32(q["s_k"])
+                       and np.float32(amax[1].item()) / np.float32(2688) == np.float32(q["s_v"]))
         out.put((rank, res))
     finally:
         dist.destroy_process_group()
@@ -90,7 +105,8 @@ def test_exchanges_reproduce_the_one_piece_layout(P):
         p.join(timeout=60)
         assert p.exitcode == 0
     for r in range(P):
-        assert results[r] == {"stats": True, "heads": True, "q": True, "o": True}, (r, results[r])
+        assert results[r] == {"stats": True, "heads": True, "q": True, "o": True,
+                              "amax": True}, (r, results[r])
 
 
 def test_shard_bounds_align_to_segments():
