@@ -185,3 +185,112 @@ def test_work_split_paths(lib, orc, H, T_c, T_q, launches):
     rows = sample_rows(T_q, n_random=16, seed=H)
     ref = orc.attention_f64(qs, Q, rows=rows)
     assert_attention_close(host_bf16_to_f64(O)[rows], ref, f"H={H} T_q={T_q}")
+
+
+def _quantized(lib, orc, K, V, ws):
+    T_c, H, _ = K.shape
+    buf = lib.ChunkBuffer(T_c, H)
+    lib.quantize_chunk(dev_bf16(K), dev_bf16(V), buf, ws)
+    return buf, orc.quantize_chunk(K, V)
+
+
+def test_largest_key_set(lib, orc):
+    """MAX_KEY_CHUNKS chunks in one call (32 sets of chunk constants: tensor
+    scales and means) match the oracle; one chunk more is refused."""
+    import torch
+    T_c, H, T_q = 64, 2, 96
+    n = lib.MAX_KEY_CHUNKS
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i in range(n + 1):
+        K = synth.k_with_offsets_bf16(300 + i, T_c, H, (T_c, H, 128))
+        V = synth.gaussian_bf16(300 + i, T_c, H, synth.T_V, (T_c, H, 128))
+        b, q = _quantized(lib, orc, K, V, ws)
+        bufs.append(b)
+        qs.append(q)
+    Q = synth.gaussian_bf16(333, T_c, H, synth.T_Q, (T_q, H, 128))
+    O = torch.empty((T_q, H, 128), dtype=torch.float32, device="cuda")
+    lib.attention(bufs[:n], dev_bf16(Q), O, ws)
+    torch.cuda.synchronize()
+    assert_attention_close(host_bf16_to_f64(O), orc.attention_f64(qs[:n], Q), f"{n} chunks")
+    with pytest.raises(lib.NvFp4KvError) as e:
+        lib.attention(bufs, dev_bf16(Q), O, ws)
+    assert e.value.status == lib.ERR_CAPACITY
+
+
+def test_zero_queries_average_the_values_full_size(lib, orc):
+    """Q = 0 makes every logit 0, so every output row is the plain mean of the
+    de-quantized V over the key set: a closed form that holds at any size,
+    checked on every row of the full one-layer workload (35,200 keys)."""
+    import torch
+    c = synth.ATTN
+    cache = lib.KVCache(1, c["H"], c["T_c"], c["S_g"], c["S_s"], c["W"])
+    want_ids = [0, 4, 7, 8, 9]
+    vsum = np.zeros((c["H"], 128), np.float64)
+    for n in range(c["appended"]):
+        if n == c["shot_start"]:
+            cache.rebind_shot_sink(n)
+        K, V, _ = synth.layer_chunk(c, 0, n)
+        cache.append(0, dev_bf16(K), dev_bf16(V))
+        if n in want_ids:
+            q = orc.quantize_chunk(K, V)
+            Vh = orc.dequantize_tensor(q["v_codes"], q["v_scales"], None, q["s_v"], c["T_c"],
+                                       c["H"], 128)
+            vsum += Vh.astype(np.float64).sum(axis=0)
+    assert cache.keyset(0) == want_ids
+    want = vsum / (len(want_ids) * c["T_c"])
+    Q = torch.zeros((c["T_c"], c["H"], 128), dtype=torch.bfloat16, device="cuda")
+    O = torch.empty((c["T_c"], c["H"], 128), dtype=torch.float32, device="cuda")
+    cache.attention(0, Q, O)
+    torch.cuda.synchronize()
+    assert cache.check_status() == lib.OK
+    ref = np.broadcast_to(want, (c["T_c"], c["H"], 128))
+    assert_attention_close(host_bf16_to_f64(O), ref, "Q = 0, every row")
+
+
+def test_growing_logits_rescale_every_tile(lib, orc):
+    """Keys whose logits grow along the key sequence by about 16 (log2 units)
+    per 128-key tile: the running maximum moves past the lazy-rescale margin on
+    every tile, so the output accumulator is rescaled each time."""
+    import torch
+    T_c, H, T_q, n = 256, 2, 130, 3
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i in range(n):
+        noise = synth.bf16_bits_to_f32(synth.gaussian_bf16(400 + i, T_c, H, synth.T_K,
+                                                           (T_c, H, 128)))
+        ramp = 6.0 * (i * T_c + np.arange(T_c, dtype=np.float32)) / (n * T_c)
+        K = synth.to_bf16_bits(ramp[:, None, None] + np.float32(0.05) * noise)
+        V = synth.gaussian_bf16(400 + i, T_c, H, synth.T_V, (T_c, H, 128))
+        b, q = _quantized(lib, orc, K, V, ws)
+        bufs.append(b)
+        qs.append(q)
+    qn = synth.bf16_bits_to_f32(synth.gaussian_bf16(410, T_c, H, synth.T_Q, (T_q, H, 128)))
+    Q = synth.to_bf16_bits(np.float32(1.0) + np.float32(0.05) * qn)
+    ref = orc.attention_f64(qs, Q)
+    for dt in (torch.float32, torch.bfloat16):
+        O = torch.empty((T_q, H, 128), dtype=dt, device="cuda")
+        lib.attention(bufs, dev_bf16(Q), O, ws)
+        torch.cuda.synchronize()
+        assert_attention_close(host_bf16_to_f64(O), ref, f"growing logits {dt}",
+                               bf16_output=dt == torch.bfloat16)
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.5])
+def test_softmax_scale_argument(lib, orc, scale):
+    import torch
+    T_c, H, T_q = 136, 3, 150
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i in range(2):
+        K = synth.k_with_offsets_bf16(500 + i, T_c, H, (T_c, H, 128))
+        V = synth.gaussian_bf16(500 + i, T_c, H, synth.T_V, (T_c, H, 128))
+        b, q = _quantized(lib, orc, K, V, ws)
+        bufs.append(b)
+        qs.append(q)
+    Q = synth.gaussian_bf16(510, T_c, H, synth.T_Q, (T_q, H, 128))
+    O = torch.empty((T_q, H, 128), dtype=torch.float32, device="cuda")
+    lib.attention(bufs, dev_bf16(Q), O, ws, softmax_scale=scale)
+    torch.cuda.synchronize()
+    assert_attention_close(host_bf16_to_f64(O), orc.attention_f64(qs, Q, scale=scale),
+                           f"softmax scale {scale}")
