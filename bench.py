@@ -513,13 +513,35 @@ class OracleSample:
                            f"scaled to the chunk ({tq_chunk:.3f} s per chunk) and prorated per "
                            f"(row, head)")}
 
+    def quantize_rates(self):
+        """The oracle's chunk quantizer alone on the slice, one thread and all
+        threads: GB/s of the chunk's algorithmic bytes (the slice's time
+        scaled to the chunk)."""
+        nbytes = quant_bytes()
+        threads = self.oracle.get_threads()
+        out = {"unit": "GB/s", "threads": threads,
+               "sample": f"{self.slice_tokens}-token slice of the 7040 x 24 x 128 chunk, "
+                         f"scaled to the chunk's {nbytes} algorithmic bytes"}
+        try:
+            for key, n in (("one_thread", 1), ("all_threads", threads)):
+                self.oracle.set_threads(n)
+                t = time.perf_counter()
+                self.oracle.quantize_chunk(self.Ks, self.Vs)
+                t_chunk = (time.perf_counter() - t) * CFG["T_c"] / self.slice_tokens
+                out[key] = nbytes / t_chunk / 1e9
+        finally:
+            self.oracle.set_threads(threads)
+        return out
+
     def baseline(self, budget_s=12.0):
         """Repeat the sample for about budget_s seconds; median value."""
         vals, t0 = [], time.perf_counter()
         while not vals or time.perf_counter() - t0 < budget_s:
             v, _, ta, tq = self.run()
             vals.append(v)
-        return self.entry(statistics.median(vals), ta, tq)
+        entry = self.entry(statistics.median(vals), ta, tq)
+        entry["quantize"] = self.quantize_rates()
+        return entry
 
 
 def run_reference(args):

@@ -277,9 +277,19 @@ nvfp4kv_status nvfp4kv_quantize_matrix(const void* X, int M, int N, int mode, vo
 
 /*
  * De-quantize a chunk back to [T_c][H][d] (device): x = decode(q) *
- * (decode(scale) * s), plus mean for K, each step one fp32 operation.
- * out_dtype: NVFP4KV_F32 or NVFP4KV_BF16 (the fp32 value rounded to nearest
- * even).  K_out or V_out may be NULL to skip that tensor.
+ * (decode(scale) * s), plus mean for K, each step one fp32 operation (the
+ * DeepRead page, Method > 推理基础设施: the cache is read back through its
+ * block and tensor scales, with K's mean restored).
+ *   in: the chunk's device pointers (16-byte aligned, as nvfp4kv_chunk_view_init
+ *       carves them); K_out, V_out: device, 16-byte aligned, T_c * H * d
+ *       elements each of out_dtype, or NULL to skip that tensor.
+ *   out_dtype: NVFP4KV_F32 or NVFP4KV_BF16 (the fp32 value rounded to nearest
+ *       even), the same for both outputs.
+ * One kernel launch for both tensors; nothing is allocated.  Errors:
+ * NVFP4KV_ERR_INVALID_ARG (null view, bad shape or dtype),
+ * NVFP4KV_ERR_UNSUPPORTED (d != 128, or no sm_100 device),
+ * NVFP4KV_ERR_ALIGNMENT, NVFP4KV_ERR_CUDA (launch failure).  Outputs must not
+ * overlap the chunk.
  */
 nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, int d,
                                   void* K_out, void* V_out, int out_dtype,
