@@ -43,6 +43,11 @@ inline TileShape tile_shape(int H) {
     return s;
 }
 
+constexpr int kMaxDevices = 64;
+// CTAs of dequant_kernel resident per SM, per device ordinal and head-block
+// width (0 = not yet asked); written by the host before the first launch.
+int g_dequant_per_sm[kMaxDevices][kTileHeads];
+
 struct DequantArgs {
     const uint8_t* codes[2];
     const uint8_t* scales[2];
@@ -233,16 +238,21 @@ nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, voi
     a.scale_stride = ts.scale_stride;
     a.buffer_bytes = ts.buffer_bytes;
     const int smem = 2 * ts.buffer_bytes;
-    // resident CTAs per SM for this buffer size (one cached answer per size)
-    static int cached_smem = -1, per_sm = 0;
-    if (smem != cached_smem) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_kernel,
-                                                          kDequantThreads, smem) != cudaSuccess)
-            per_sm = 0;
-        cached_smem = per_sm > 0 ? smem : -1;
+    // resident CTAs per SM for this buffer size, asked once per device and size
+    // (the buffer size depends on min(H, kTileHeads) only)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4KV_ERR_CUDA;
+    const int hb = H < kTileHeads ? H : kTileHeads;
+    int& per_sm = g_dequant_per_sm[dev][hb - 1];
+    if (per_sm == 0 &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_kernel, kDequantThreads,
+                                                       smem) != cudaSuccess ||
+         per_sm < 1)) {
+        per_sm = 0;
+        return NVFP4KV_ERR_CUDA;
     }
     const int sms = sm_count_cached();
-    if (per_sm <= 0 || sms <= 0) return NVFP4KV_ERR_CUDA;
+    if (sms <= 0) return NVFP4KV_ERR_CUDA;
     // as many rounds as the resident CTAs need, then the fewest CTAs that
     // still finish in that many rounds, so that every CTA gets the same count
     const long units = (long)a.n_tensors * a.tiles_per_tensor;
