@@ -58,7 +58,7 @@ NCU_TRAFFIC = {
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
                  "6a8cb7ce1a56316e2dad4dd9c3ecd74d349d1a1ea48f29dcccb9dfda8cd02dec", 97600000),
     "dequantize": ("sink_window_video_b200/csrc/dequant.cu",
-                   "abbdbf999d98f485296aa8637dda0439dda52de694237ef5f4cb6239b7ebf0f9", 51689728),
+                   "7dd04c898e146642244e3c647f75a4c6d746e2fad0c7c310a2255267bb2fd8f6", 51334400),
 }
 
 

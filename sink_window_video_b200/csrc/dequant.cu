@@ -57,6 +57,7 @@ struct DequantArgs {
     int which[2];                       // tensor of each of the n_tensors slots
     int n_tensors, T, H, n_hb, tiles_per_tensor, out_bf16;
     int code_stride, scale_stride, buffer_bytes;
+    float one;                          // 1, as a run-time value (see decode8)
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -77,27 +78,24 @@ __device__ __forceinline__ float2 f16x2_to_f32x2_exact(uint32_t h2) {
 }
 
 // Eight decoded elements: x = RN(code * D) (+ mean, one more RN), each step
-// one IEEE fp32 operation.
-__device__ __forceinline__ void decode8(uint32_t q, float D, const float* mean, float* x) {
+// one IEEE fp32 operation, on float pairs.  The mean is added as
+// fma(mean, one, x) with one = 1 held in a run-time value: the same single
+// rounding, and a form the compiler cannot merge with the product before it.
+__device__ __forceinline__ void decode8(uint32_t q, float D, const float* mean, float one,
+                                        float2* x) {
     uint32_t hq[4];
     cvt_e2m1x8_to_f16x2(q, hq);
+    const float2 D2 = make_float2(D, D);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 c = f16x2_to_f32x2_exact(hq[j]);
-        x[2 * j] = __fmul_rn(c.x, D);
-        x[2 * j + 1] = __fmul_rn(c.y, D);
-    }
+    for (int j = 0; j < 4; ++j) x[j] = __fmul2_rn(f16x2_to_f32x2_exact(hq[j]), D2);
     if (mean) {
         const float4 m0 = __ldg(reinterpret_cast<const float4*>(mean));
         const float4 m1 = __ldg(reinterpret_cast<const float4*>(mean) + 1);
-        x[0] = __fadd_rn(x[0], m0.x);
-        x[1] = __fadd_rn(x[1], m0.y);
-        x[2] = __fadd_rn(x[2], m0.z);
-        x[3] = __fadd_rn(x[3], m0.w);
-        x[4] = __fadd_rn(x[4], m1.x);
-        x[5] = __fadd_rn(x[5], m1.y);
-        x[6] = __fadd_rn(x[6], m1.z);
-        x[7] = __fadd_rn(x[7], m1.w);
+        const float2 ONE = make_float2(one, one);
+        x[0] = __ffma2_rn(make_float2(m0.x, m0.y), ONE, x[0]);
+        x[1] = __ffma2_rn(make_float2(m0.z, m0.w), ONE, x[1]);
+        x[2] = __ffma2_rn(make_float2(m1.x, m1.y), ONE, x[2]);
+        x[3] = __ffma2_rn(make_float2(m1.z, m1.w), ONE, x[3]);
     }
 }
 
@@ -150,7 +148,7 @@ __device__ __forceinline__ void prefetch_tile(const DequantArgs& a, const Tile& 
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(kDequantThreads) dequant_kernel(const DequantArgs a) {
+__global__ void __launch_bounds__(kDequantThreads, 6) dequant_kernel(const DequantArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int units = a.n_tensors * a.tiles_per_tensor;
     int b = 0;
@@ -181,22 +179,22 @@ __global__ void __launch_bounds__(kDequantThreads) dequant_kernel(const DequantA
         for (int c = threadIdx.x; c < n_pieces; c += kDequantThreads) {
             const uint32_t q = *reinterpret_cast<const uint32_t*>(cs + tt * a.code_stride + h * 64 + g * 4);
             const float D = __fmul_rn(e4m3_to_f32(ss[tt * a.scale_stride + h * 8 + (g >> 1)]), s);
-            float x[8];
-            decode8(q, D, mean ? mean + (t.h0 + h) * kHeadDim + g * 8 : nullptr, x);
+            float2 x[4];
+            decode8(q, D, mean ? mean + (t.h0 + h) * kHeadDim + g * 8 : nullptr, a.one, x);
             const size_t o = ((size_t)(t.t0 + tt) * a.H + t.h0 + h) * kHeadDim + g * 8;
             if (a.out_bf16) {
                 uint32_t wv[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    __nv_bfloat162 p = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+                    __nv_bfloat162 p = __floats2bfloat162_rn(x[j].x, x[j].y);
                     wv[j] = *reinterpret_cast<uint32_t*>(&p);
                 }
                 __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + o),
                        make_uint4(wv[0], wv[1], wv[2], wv[3]));
             } else {
                 float4* p = reinterpret_cast<float4*>(static_cast<float*>(out) + o);
-                __stcs(p, make_float4(x[0], x[1], x[2], x[3]));
-                __stcs(p + 1, make_float4(x[4], x[5], x[6], x[7]));
+                __stcs(p, make_float4(x[0].x, x[0].y, x[1].x, x[1].y));
+                __stcs(p + 1, make_float4(x[2].x, x[2].y, x[3].x, x[3].y));
             }
             tt += dtt;
             h += dh;
@@ -233,6 +231,7 @@ nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, voi
     a.n_hb = (H + kTileHeads - 1) / kTileHeads;
     a.tiles_per_tensor = ((T + kTileTokens - 1) / kTileTokens) * a.n_hb;
     a.out_bf16 = out_dtype == NVFP4KV_BF16 ? 1 : 0;
+    a.one = 1.0f;
     const TileShape ts = tile_shape(H);
     a.code_stride = ts.code_stride;
     a.scale_stride = ts.scale_stride;
