@@ -294,3 +294,32 @@ def test_softmax_scale_argument(lib, orc, scale):
     torch.cuda.synchronize()
     assert_attention_close(host_bf16_to_f64(O), orc.attention_f64(qs, Q, scale=scale),
                            f"softmax scale {scale}")
+
+
+def test_repeated_calls_are_bit_identical(lib):
+    """The same call twice writes the same bytes, through the split-tail path
+    (partial results merged by a second kernel) and in both output types: the
+    accumulation order is fixed, so a replica on another GPU reproduces a
+    one-GPU run exactly."""
+    import torch
+    T_c, H, T_q = 600, 3, 500
+    assert lib.attention_launches(2, T_c, H, T_q) == 2
+    ws = lib.new_workspace(T_c, H)
+    bufs = []
+    for i in range(2):
+        K = synth.k_with_offsets_bf16(600 + i, T_c, H, (T_c, H, 128))
+        V = synth.gaussian_bf16(600 + i, T_c, H, synth.T_V, (T_c, H, 128))
+        b = lib.ChunkBuffer(T_c, H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), b, ws)
+        bufs.append(b)
+    Q = dev_bf16(synth.gaussian_bf16(610, T_c, H, synth.T_Q, (T_q, H, 128)))
+    for dt in (torch.float32, torch.bfloat16):
+        outs = []
+        for _ in range(2):
+            O = torch.full((T_q, H, 128), float("nan"), dtype=dt, device="cuda")
+            lib.attention(bufs, Q, O, ws)
+            outs.append(O)
+        torch.cuda.synchronize()
+        assert lib.workspace_status(ws) == lib.OK
+        assert torch.equal(outs[0].view(torch.int16 if dt == torch.bfloat16 else torch.int32),
+                           outs[1].view(torch.int16 if dt == torch.bfloat16 else torch.int32))
