@@ -608,12 +608,15 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": r["ms_total"] / K,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded SplitMix64 + Box-Muller, 5B video DiT shapes)",
             "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": CFG["T_c"],
                        "keys": keys_per_step(), "heads": CFG["H"], "head_dim": CFG["d"],
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs rotate over 4 sets of K,V,Q (520 MB) > 126 MB L2"},
+                       "l2": "inputs rotate over 4 sets of K,V,Q (520 MB) > 126 MB L2",
+                       "arithmetic": "attention MMAs on fp16 operands (the de-quantized cache "
+                                     "exactly; bf16 Q scaled by 2^-e), fp32 accumulation and "
+                                     "softmax; quantizer in fp32"},
             "roofline": {"bound": "tensor", "kernel": "sink_window_attention",
                          "achieved": attn_tf, "peak": tpeak, "unit": "TFLOP/s",
                          "frac": attn_tf / tpeak, "traffic": ncu_traffic("attention"),
