@@ -60,6 +60,8 @@ def lib():
         L.oracle_keyset.argtypes = [ctypes.c_int64, i32, i32, i32, ctypes.c_int64, vp]
         L.oracle_attention_f64.argtypes = [vp, i32, i32, i32, vp, i32, vp, i32,
                                            ctypes.c_double, vp]
+        L.oracle_attention_f64_fq.argtypes = [vp, i32, i32, i32, vp, i32, vp, i32,
+                                              ctypes.c_double, vp]
         L.oracle_chunk_payload_bytes.restype = sz
         L.oracle_chunk_payload_bytes.argtypes = [i32, i32, i32]
         L.oracle_quantize_matrix.restype = i32
@@ -224,12 +226,7 @@ def keyset(n: int, S_g: int, S_s: int, W: int, s_begin: int):
 
 # ---------------------------------------------------------------- attention
 
-def attention_f64(chunks, Q: np.ndarray, rows=None, scale: float = 0.0) -> np.ndarray:
-    """Float64 attention of Q [T_q, H, d] (bf16 bits) over the listed quantized
-    chunks (dicts as returned by quantize_chunk, in key order).  rows: query rows
-    to evaluate (None = all).  Returns [n_rows, H, d] float64."""
-    Q = np.ascontiguousarray(Q, dtype=np.uint16)
-    T_q, H, d = Q.shape
+def _chunk_array(chunks):
     keep = []
     arr = (OracleChunk * max(1, len(chunks)))()
     for i, c in enumerate(chunks):
@@ -238,6 +235,12 @@ def attention_f64(chunks, Q: np.ndarray, rows=None, scale: float = 0.0) -> np.nd
         keep.append(parts)
         arr[i] = OracleChunk(*(p.ctypes.data for p in parts), float(c["s_k"]),
                              float(c["s_v"]), int(c["k_codes"].shape[1]))
+    return arr, keep
+
+
+def _attention(fn, chunks, Q, rows, scale):
+    T_q, H, d = Q.shape
+    arr, keep = _chunk_array(chunks)
     if rows is None:
         rows_arr = None
         n_rows = T_q
@@ -247,6 +250,40 @@ def attention_f64(chunks, Q: np.ndarray, rows=None, scale: float = 0.0) -> np.nd
     out = np.zeros((n_rows, H, d), np.float64)
     if not (scale > 0):
         scale = 1.0 / math.sqrt(d)
-    lib().oracle_attention_f64(arr, len(chunks), H, d, _ptr(Q), T_q, _ptr(rows_arr), n_rows,
-                               float(scale), _ptr(out))
+    fn(arr, len(chunks), H, d, _ptr(Q), T_q, _ptr(rows_arr), n_rows, float(scale), _ptr(out))
+    del keep
     return out
+
+
+def attention_f64(chunks, Q: np.ndarray, rows=None, scale: float = 0.0) -> np.ndarray:
+    """Float64 attention of Q [T_q, H, d] (bf16 bits) over the listed quantized
+    chunks (dicts as returned by quantize_chunk, in key order).  rows: query rows
+    to evaluate (None = all).  Returns [n_rows, H, d] float64."""
+    Q = np.ascontiguousarray(Q, dtype=np.uint16)
+    return _attention(lib().oracle_attention_f64, chunks, Q, rows, scale)
+
+
+def attention_f64_fq(chunks, Qf: np.ndarray, rows=None, scale: float = 0.0) -> np.ndarray:
+    """attention_f64 for queries given as fp32 values [T_q, H, d]."""
+    Qf = np.ascontiguousarray(Qf, dtype=np.float32)
+    return _attention(lib().oracle_attention_f64_fq, chunks, Qf, rows, scale)
+
+
+def quantize_queries(Q: np.ndarray):
+    """NVFP4 of the queries for an FP4-operand S = Q K^T ("2605-LongLive2"
+    DeepRead page, Method > 推理基础设施: W4A4 on Blackwell, FP4 GEMMs in place of
+    BF16 ones; Method > 训练基础设施: activations in 1D blocks): Q [T_q, H, d]
+    (bf16 bits) as the matrix [T_q * H, d], 16-element blocks along d -- the
+    contraction -- with Four-Over-Six and one FP32 tensor scale (quantize_matrix,
+    MATRIX_1D).  Returns (the quantize_matrix dict, Q_hat [T_q, H, d] fp32)."""
+    Q = np.ascontiguousarray(Q, dtype=np.uint16)
+    T_q, H, d = Q.shape
+    q = quantize_matrix(Q.reshape(T_q * H, d), MATRIX_1D)
+    return q, dequantize_matrix(q, MATRIX_1D).reshape(T_q, H, d)
+
+
+def attention_f64_fp4q(chunks, Q: np.ndarray, rows=None, scale: float = 0.0) -> np.ndarray:
+    """Float64 attention with the queries replaced by their NVFP4 reconstruction
+    (quantize_queries): the reference for an FP4-operand Q K^T over the cache."""
+    _, Qh = quantize_queries(Q)
+    return attention_f64_fq(chunks, Qh, rows, scale)

@@ -474,9 +474,11 @@ static double dq_elem(const uint8_t* codes, const uint8_t* scales, const float* 
  *   out:  [n_rows][H][d] double
  * Loops heads outermost; keys of one head are expanded to double once.
  */
-void oracle_attention_f64(const oracle_chunk* chunks, int n_chunks, int H, int d,
-                          const uint16_t* Q, int T_q, const int* rows, int n_rows,
-                          double scale, double* out) {
+/* The attention of either Q form: Qb (bf16 bits) or Qf (fp32 values), the
+ * other NULL; both are widened exactly to float64. */
+static void attention_core(const oracle_chunk* chunks, int n_chunks, int H, int d,
+                           const uint16_t* Qb, const float* Qf, int T_q, const int* rows,
+                           int n_rows, double scale, double* out) {
     int L = 0;
     for (int k = 0; k < n_chunks; ++k) L += chunks[k].T;
     if (L == 0) return;
@@ -500,8 +502,10 @@ void oracle_attention_f64(const oracle_chunk* chunks, int n_chunks, int H, int d
             int i = rows ? rows[r] : r;
             double* q = (double*)malloc((size_t)d * sizeof(double));
             double* p = (double*)malloc((size_t)L * sizeof(double));
-            for (int c = 0; c < d; ++c)
-                q[c] = (double)oracle_bf16_to_f32(Q[((size_t)i * H + h) * d + c]);
+            for (int c = 0; c < d; ++c) {
+                const size_t e = ((size_t)i * H + h) * d + c;
+                q[c] = Qb ? (double)oracle_bf16_to_f32(Qb[e]) : (double)Qf[e];
+            }
             double mx = -INFINITY;
             for (int jj = 0; jj < L; ++jj) {
                 double acc = 0.0;
@@ -537,6 +541,23 @@ size_t oracle_chunk_payload_bytes(int T, int H, int d) {
 /* ------------------------------------------------------------------------ */
 /* Array helpers for the test harness (loops over the scalar functions).     */
 /* ------------------------------------------------------------------------ */
+
+void oracle_attention_f64(const oracle_chunk* chunks, int n_chunks, int H, int d,
+                          const uint16_t* Q, int T_q, const int* rows, int n_rows,
+                          double scale, double* out) {
+    attention_core(chunks, n_chunks, H, d, Q, NULL, T_q, rows, n_rows, scale, out);
+}
+
+/* The same attention for queries given as fp32 values: used with Q replaced by
+ * its NVFP4 reconstruction, the FP4-operand form of S = Q K^T ("2605-LongLive2"
+ * DeepRead page, Method > 推理基础设施: on Blackwell the generator runs W4A4,
+ * FP4 GEMMs in place of BF16 ones; Method > 训练基础设施: activations take 1D
+ * blocks along the contraction). */
+void oracle_attention_f64_fq(const oracle_chunk* chunks, int n_chunks, int H, int d,
+                             const float* Qf, int T_q, const int* rows, int n_rows,
+                             double scale, double* out) {
+    attention_core(chunks, n_chunks, H, d, NULL, Qf, T_q, rows, n_rows, scale, out);
+}
 
 void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
 int oracle_get_threads(void) { return omp_get_max_threads(); }
