@@ -73,3 +73,22 @@ def test_degenerate_and_extreme_inputs(lib, orc, mode):
     ws = None
     for X_, what in cases:
         ws = _check(lib, orc, X_, mode, ws, what)
+
+
+def test_query_quantization_at_the_layer_shape(lib, orc):
+    """The first step of an FP4-operand Q K^T: the layer's queries [7040, 24, 128]
+    as the matrix [7040 * 24, 128], 16-element blocks along d, bit-exact against
+    the oracle's quantize_queries (codes, scale bytes, tensor scale)."""
+    import torch
+    T_q, H = 7040, 24
+    Q = synth.gaussian_bf16(800, 0, 0, synth.T_Q, (T_q, H, 128))
+    ws = lib.new_matrix_workspace()
+    out = lib.MatrixBuffer(T_q * H, 128, 1)
+    lib.quantize_matrix(_dev(Q).view(T_q * H, 128), out, ws)
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    got = out.to_host()
+    ref, _ = orc.quantize_queries(Q)
+    assert np.float32(got["s"]) == np.float32(ref["s"])
+    assert np.array_equal(got["scales"], ref["scales"])
+    assert np.array_equal(got["codes"], ref["codes"])
