@@ -575,6 +575,55 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ main
 
+def build_line(args, r, world, peaks, peak_src):
+    """The JSON line of our arm from run_ours' measurements r (every key but
+    cpu_baseline, which main adds)."""
+    K = args.steps
+    value = whole_job_rate(attn_flops(), K, world, r["ms_total"]) / 1e12
+    attn_tf = attn_flops() / (r["ms_attn"] / 1e3) / 1e12
+    quant_gbs = quant_bytes() / (r["ms_quant"] / 1e3) / 1e9
+    tpeak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": r["ms_total"] / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded SplitMix64 + Box-Muller, 5B video DiT shapes)",
+        "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": CFG["T_c"],
+                   "keys": keys_per_step(), "heads": CFG["H"], "head_dim": CFG["d"],
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs rotate over 4 sets of K,V,Q (520 MB) > 126 MB L2",
+                   "arithmetic": "attention MMAs on fp16 operands (the de-quantized cache "
+                                 "exactly; bf16 Q scaled by 2^-e), fp32 accumulation and "
+                                 "softmax; quantizer in fp32"},
+        "roofline": {"bound": "tensor", "kernel": "sink_window_attention",
+                     "achieved": attn_tf, "peak": tpeak, "unit": "TFLOP/s",
+                     "frac": attn_tf / tpeak, "traffic": ncu_traffic("attention"),
+                     "peak_source": f"{peak_src} bf16 sustained"},
+        "quantize": {"kernel": "nvfp4kv_quantize_chunk", "bound": "hbm",
+                     "achieved": quant_gbs, "peak": hpeak, "unit": "GB/s",
+                     "frac": quant_gbs / hpeak, "bytes_per_launch": quant_bytes(),
+                     "traffic": ncu_traffic("quantize"),
+                     "ms_per_launch": r["ms_quant"], "peak_source": f"{peak_src} hbm"},
+        "attention": {"ms_per_launch": r["ms_attn"], "flops_per_launch": attn_flops(),
+                      "tflops": attn_tf},
+        "gpu_launches": K * (1 + r["attn_launches"]),
+        "clocks": r["clocks"],
+    }
+    if r["e2e_ms"] is not None:
+        n = CFG["T_c"] * CFG["H"] * CFG["d"]
+        line["e2e"] = {"value": attn_flops() * world / (r["e2e_ms"] / 1e3) / 1e12,
+                       "unit": "TFLOP/s", "h2d_bytes_per_step": 3 * n * 2,
+                       "d2h_bytes_per_step": n * 2, "ms_per_step": r["e2e_ms"]}
+    if r["rollouts"] is not None:
+        line["rollouts"] = r["rollouts"]
+    if r["matrix"] is not None:
+        line["matrix_quantize"] = r["matrix"]
+    if r["dequant"] is not None:
+        line["dequantize"] = r["dequant"]
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -599,49 +648,7 @@ def main():
     r = run_ours(args, rank, world, local)
     peaks, peak_src = load_peaks()
     if rank == 0:
-        K = args.steps
-        value = whole_job_rate(attn_flops(), K, world, r["ms_total"]) / 1e12
-        attn_tf = attn_flops() / (r["ms_attn"] / 1e3) / 1e12
-        quant_gbs = quant_bytes() / (r["ms_quant"] / 1e3) / 1e9
-        tpeak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-        hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": r["ms_total"] / K,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-            "data": "synthetic (seeded SplitMix64 + Box-Muller, 5B video DiT shapes)",
-            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": CFG["T_c"],
-                       "keys": keys_per_step(), "heads": CFG["H"], "head_dim": CFG["d"],
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs rotate over 4 sets of K,V,Q (520 MB) > 126 MB L2",
-                       "arithmetic": "attention MMAs on fp16 operands (the de-quantized cache "
-                                     "exactly; bf16 Q scaled by 2^-e), fp32 accumulation and "
-                                     "softmax; quantizer in fp32"},
-            "roofline": {"bound": "tensor", "kernel": "sink_window_attention",
-                         "achieved": attn_tf, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": attn_tf / tpeak, "traffic": ncu_traffic("attention"),
-                         "peak_source": f"{peak_src} bf16 sustained"},
-            "quantize": {"kernel": "nvfp4kv_quantize_chunk", "bound": "hbm",
-                         "achieved": quant_gbs, "peak": hpeak, "unit": "GB/s",
-                         "frac": quant_gbs / hpeak, "bytes_per_launch": quant_bytes(),
-                         "traffic": ncu_traffic("quantize"),
-                         "ms_per_launch": r["ms_quant"], "peak_source": f"{peak_src} hbm"},
-            "attention": {"ms_per_launch": r["ms_attn"], "flops_per_launch": attn_flops(),
-                          "tflops": attn_tf},
-            "gpu_launches": K * (1 + r["attn_launches"]),
-            "clocks": r["clocks"],
-        }
-        if r["e2e_ms"] is not None:
-            n = CFG["T_c"] * CFG["H"] * CFG["d"]
-            line["e2e"] = {"value": attn_flops() * world / (r["e2e_ms"] / 1e3) / 1e12,
-                           "unit": "TFLOP/s", "h2d_bytes_per_step": 3 * n * 2,
-                           "d2h_bytes_per_step": n * 2, "ms_per_step": r["e2e_ms"]}
-        if r["rollouts"] is not None:
-            line["rollouts"] = r["rollouts"]
-        if r["matrix"] is not None:
-            line["matrix_quantize"] = r["matrix"]
-        if r["dequant"] is not None:
-            line["dequantize"] = r["dequant"]
+        line = build_line(args, r, world, peaks, peak_src)
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = OracleSample(rows=args.ref_rows).baseline()
         print(json.dumps(line))
