@@ -12,7 +12,9 @@
  *         Method > 训练基础设施 (NVFP4 training: E2M1 values, block FP8 E4M3
  *         scale, tensor FP32 scale; scale search over targets 6 and 4),
  *         Method > 推理基础设施 (parallel KV quantization: chunk level,
- *         K-smoothing, micro-block NVFP4, (9/8)T_c*H*d bytes),
+ *         K-smoothing, micro-block NVFP4, (9/8)T_c*H*d bytes; W4A4 on
+ *         Blackwell, FP4 GEMMs in place of BF16 ones -- the attention over
+ *         fp32 queries serves the FP4-query form of S = Q K^T),
  *         Method > 算法层设计 (Multi-Shot Attention Sink: A_g, A_s,
  *         K_eff(t) = A_g u A_s u KV[t-W,t), de-duplication, two pointers).
  *   [TN]  "LongLive-2.0: Infrastruttura Parallela NVFP4 per Video Lunghi"
