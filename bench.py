@@ -575,6 +575,13 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ main
 
+def wants_cpu_baseline(args, world):
+    """The oracle's timing runs on rank 0 of a one-GPU run only: a bounded
+    sample on the host cores, which a multi-GPU run would only keep the other
+    ranks waiting for."""
+    return world == 1 and not args.no_cpu_baseline
+
+
 def build_line(args, r, world, peaks, peak_src):
     """The JSON line of our arm from run_ours' measurements r (every key but
     cpu_baseline, which main adds)."""
@@ -649,7 +656,7 @@ def main():
     peaks, peak_src = load_peaks()
     if rank == 0:
         line = build_line(args, r, world, peaks, peak_src)
-        if not args.no_cpu_baseline:
+        if wants_cpu_baseline(args, world):
             line["cpu_baseline"] = OracleSample(rows=args.ref_rows).baseline()
         print(json.dumps(line))
     barrier(world)

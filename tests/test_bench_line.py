@@ -54,3 +54,12 @@ def test_line_without_optional_parts():
     for k in ("e2e", "rollouts", "matrix_quantize", "dequantize"):
         assert k not in line
     json.dumps(line)
+
+
+def test_cpu_baseline_only_in_one_gpu_runs():
+    import bench
+    on = types.SimpleNamespace(no_cpu_baseline=False)
+    off = types.SimpleNamespace(no_cpu_baseline=True)
+    assert bench.wants_cpu_baseline(on, 1)
+    assert not bench.wants_cpu_baseline(on, 2)
+    assert not bench.wants_cpu_baseline(off, 1)
