@@ -66,6 +66,7 @@ def load():
         "nvfp4kv_workspace_init": (st, [vp, sz, vp]),
         "nvfp4kv_workspace_status": (st, [vp, vp]),
         "nvfp4kv_quantize_chunk": (st, [vp, vp, i32, i32, i32, cv, vp, vp]),
+        "nvfp4kv_quantize_chunk_noalloc": (st, [vp, vp, i32, i32, i32, cv, vp]),
         "nvfp4kv_dequantize": (st, [cv, i32, i32, i32, vp, vp, i32, vp]),
         "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp]),
         "nvfp4kv_attention_launches": (i32, [i32, i32, i32, i32, i32]),
@@ -332,6 +333,15 @@ def quantize_chunk(K, V, out: ChunkBuffer, ws, stream=None):
     T, H, d = K.shape
     _check(load().nvfp4kv_quantize_chunk(_ptr(K), _ptr(V), T, H, d, ctypes.byref(out.view),
                                          _ptr(ws), _stream(stream)), "nvfp4kv_quantize_chunk")
+
+
+def quantize_chunk_noalloc(K, V, out: ChunkBuffer, stream=None):
+    """quantize_chunk without a workspace: the library's compiled-in scratch
+    (chunks whose scratch exceeds it are refused with ERR_CAPACITY)."""
+    T, H, d = K.shape
+    _check(load().nvfp4kv_quantize_chunk_noalloc(_ptr(K), _ptr(V), T, H, d,
+                                                 ctypes.byref(out.view), _stream(stream)),
+           "nvfp4kv_quantize_chunk_noalloc")
 
 
 def dequantize(chunk: ChunkBuffer, K_out=None, V_out=None, stream=None):

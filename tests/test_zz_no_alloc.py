@@ -3,7 +3,8 @@ allocate device memory (engines that own all GPU memory and give plugins no
 scratch, real-time loops that must not risk cudaMalloc's synchronization).  It
 keeps its scratch in an array compiled into the library instead of a caller
 workspace.  Checked through the C ABI against nvfp4kv_quantize_chunk (the
-workspace entry point), bit for bit, on two calls in a row; this file is
+workspace entry point), bit for bit, on two calls in a row (through the
+Python binding), and its refusals through the raw C ABI; this file is
 collected last so that a failure here comes after every other test ran."""
 import ctypes
 
@@ -32,8 +33,6 @@ def _parts(buf):
 
 def test_noalloc_matches_workspace_entry_point_twice(lib):
     import torch
-    fn = _entry(lib)
-    stream = torch.cuda.current_stream().cuda_stream
     inputs = [synth.quant_chunk(0), synth.layer_chunk(synth.MULTISHOT, 0, 3)[:2]]
     for call, (K, V) in enumerate(inputs):
         T, H, d = K.shape
@@ -42,8 +41,7 @@ def test_noalloc_matches_workspace_entry_point_twice(lib):
         ws = lib.new_workspace(T, H, d)
         lib.quantize_chunk(Kd, Vd, ref, ws)
         got = lib.ChunkBuffer(T, H, d)
-        st = fn(Kd.data_ptr(), Vd.data_ptr(), T, H, d, ctypes.byref(got.view), stream)
-        assert st == lib.OK, f"call {call}: status {st}"
+        lib.quantize_chunk_noalloc(Kd, Vd, got)          # raises on a status other than OK
         torch.cuda.synchronize()
         assert lib.workspace_status(ws) == lib.OK
         a, b = _parts(got), _parts(ref)
