@@ -153,14 +153,20 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
  * are refused with NVFP4KV_ERR_CAPACITY before any device work (H = 24,
  * d = 128 allows T_c up to 10,816).  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture.  Every call
+ * current; make that first call before any stream capture.  The address is
+ * kept for the life of the process: do not use this entry point across a
+ * device reset (cudaDeviceReset, or a primary context destroyed and created
+ * again), which reloads the library's module at a new address; a call that
+ * fails with NVFP4KV_ERR_CUDA drops the kept address, so the next call looks
+ * it up again.  Every call
  * clears the barrier and status words on `stream` and then reuses the same
  * array, so calls that overlap on the GPU (other streams, other threads)
  * race; the array keeps the last call's contents.  A kernel-side timeout is
  * not reported here; use nvfp4kv_quantize_chunk with a workspace to read it.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
- * Output, arguments and other errors are those of nvfp4kv_quantize_chunk,
- * bit for bit.
+ * Output, and the status returned for every argument error, are those of
+ * nvfp4kv_quantize_chunk (its checks run first, in its order, the workspace
+ * left out); NVFP4KV_ERR_CAPACITY follows them.
  */
 nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const void* V, int T_c, int H,
                                               int d, const nvfp4kv_chunk_view* out,
@@ -420,7 +426,8 @@ nvfp4kv_status kvcache_check_status(kvcache* cache, nvfp4kv_stream_t stream);
  * op 0: E2M1 code of each fp32 input (one code per output byte),
  * op 1: E4M3 byte of each fp32 input, op 2: fp32 value of each E2M1 code,
  * op 3: fp32 value of each E4M3 byte, op 4: the fp32 quotient x/D that the
- * quantizer forms for a pair (in[2i] = x, in[2i+1] = D > 0).
+ * quantizer forms for a pair (in[2i] = x, in[2i+1] = D > 0), op 5: 2^x
+ * by the attention softmax's polynomial on the FMA pipe (for x >= -126).
  * in/out are device arrays of n elements (op 4: n quotients from 2n inputs).
  */
 nvfp4kv_status nvfp4kv_check_formats(int op, const void* in, void* out, size_t n,

@@ -124,21 +124,21 @@ bool have_sm100() {
 }  // namespace
 
 namespace nvfp4kv {
+nvfp4kv_status check_quantize_chunk_args(const void* K, const void* V, int T_c, int H, int d,
+                                         const nvfp4kv_chunk_view* out, const void* ws,
+                                         bool need_ws) {
+    if (!K || !V || !out || (need_ws && !ws) || !valid_shape(T_c, H, d) || !view_ok(*out))
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned16(K) || !aligned16(V) || (need_ws && !aligned256(ws)))
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return NVFP4KV_OK;
+}
+
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c, int H,
                                 const void* Q, int T_q, void* O, int o_dtype, float softmax_scale,
                                 void* ws, cudaStream_t stream) {
-    static const int which = [] {
-        const char* e = std::getenv("NVFP4KV_ATTENTION_KERNEL");
-        if (e != nullptr && std::strcmp(e, "mma") == 0) return 1;
-        if (e != nullptr && std::strcmp(e, "tc1") == 0) return 2;
-        return 0;
-    }();
-    if (which == 1)
-        return launch_attention_mma(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
-                                    stream);
-    if (which == 2)
-        return launch_attention_tc(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
-                                   ws, stream);
     return launch_attention_ws(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale, ws,
                                stream);
 }
@@ -165,8 +165,6 @@ int nvfp4kv_attention_launches(int n_chunks, int T_c, int H, int d, int T_q) {
     if (!valid_shape(T_c, H, d) || n_chunks < 1 || n_chunks > NVFP4KV_MAX_KEY_CHUNKS ||
         T_q <= 0)
         return 0;
-    const char* e = std::getenv("NVFP4KV_ATTENTION_KERNEL");
-    if (e != nullptr && (std::strcmp(e, "mma") == 0 || std::strcmp(e, "tc1") == 0)) return 1;
     const AttnPlan p = attention_plan(n_chunks, T_c, H, T_q, ws_layout(T_c, H).apart_pairs);
     return p.n_tail > 0 ? 2 : 1;
 }
@@ -200,11 +198,8 @@ nvfp4kv_status nvfp4kv_workspace_status(void* ws, nvfp4kv_stream_t stream) {
 nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int H, int d,
                                       const nvfp4kv_chunk_view* out, void* ws,
                                       nvfp4kv_stream_t stream) {
-    if (!K || !V || !out || !ws || !valid_shape(T_c, H, d) || !view_ok(*out))
-        return NVFP4KV_ERR_INVALID_ARG;
-    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
-    if (!aligned16(K) || !aligned16(V) || !aligned256(ws)) return NVFP4KV_ERR_ALIGNMENT;
-    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    const nvfp4kv_status st = check_quantize_chunk_args(K, V, T_c, H, d, out, ws, true);
+    if (st != NVFP4KV_OK) return st;
     return launch_quantize(K, V, T_c, H, *out, ws, (cudaStream_t)stream);
 }
 
@@ -322,7 +317,7 @@ nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
 
 nvfp4kv_status nvfp4kv_check_formats(int op, const void* in, void* out, size_t n,
                                      nvfp4kv_stream_t stream) {
-    if (!in || !out || op < 0 || op > 4) return NVFP4KV_ERR_INVALID_ARG;
+    if (!in || !out || op < 0 || op > 5) return NVFP4KV_ERR_INVALID_ARG;
     if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
     return launch_check_formats(op, in, out, n, (cudaStream_t)stream);
 }

@@ -30,7 +30,8 @@ struct Control {
     unsigned bar_count;   // grid barrier: CTAs arrived at the current barrier
     unsigned bar_gen;     // grid barrier: generation, bumped by the last arrival
     unsigned diag[4];     // first wait that gave up: site, block (x | y << 16), step, phase
-    unsigned pad0[2];
+    unsigned test_flags;  // test hooks, 0 in normal use (bit 0: see attention_ws.cu)
+    unsigned pad0;
     unsigned long long stamp[8];   // %globaltimer at CTA 0's phase boundaries (diagnostics)
     unsigned pad[38];
 };
@@ -185,6 +186,29 @@ __device__ __forceinline__ float div_markstein(float x, float D, float r) {
     float q0 = __fmul_rn(x, r);
     float e = __fmaf_rn(-q0, D, x);
     return __fmaf_rn(e, r, q0);
+}
+
+// 2^x for a pair on the FMA and integer pipes (in the attention's softmax the
+// special-function unit is shared by two warps per sub-partition and is the
+// scarcer resource):
+// n = round(x) by adding and subtracting 1.5*2^23, f = x - n in [-1/2, 1/2],
+// 2^f by a cubic (least-squares fit on relative error, max 7.5e-5), and 2^n
+// added to the exponent field.  x is clamped to -126 so 2^n stays normal;
+// inputs here are at most 8 (the lazy-max bound).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+    float2 p = __ffma2_rn(make_float2(0.055170949548482895f, 0.055170949548482895f), f,
+                          make_float2(0.2426096349954605f, 0.2426096349954605f));
+    p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = __ffma2_rn(p, f, make_float2(0.9999281764030457f, 0.9999281764030457f));
+    float2 r;
+    r.x = __int_as_float(__float_as_int(p.x) + ((__float_as_int(t.x) - 0x4B400000) << 23));
+    r.y = __int_as_float(__float_as_int(p.y) + ((__float_as_int(t.y) - 0x4B400000) << 23));
+    return r;
 }
 
 }  // namespace nvfp4kv

@@ -16,11 +16,11 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Attention work split (see launch_attention_ws): the 256-row query blocks
 // that do not fill a whole wave of CTAs are split into up to kMaxSplit key
-// ranges, whose partial results (per row: 128 fp32 outputs, the running max
+// ranges, whose partial results (per row: 128 fp32 outputs, the two running maxima
 // and the row sum) go to the workspace and are merged by a second kernel.
 constexpr int kMaxTailPairs = 160;   // more than one wave never remains
 constexpr int kMaxSplit = 8;
-constexpr int kPartialFloats = 132;  // per row: O[128], m, l, 2 pad (16-byte rows)
+constexpr int kPartialFloats = 132;  // per row: O[128], m_o, m_l, l, 1 pad (16-byte rows)
 
 // Workspace layout for chunks of T tokens and H heads (d = 128):
 //   [0, 256)  Control (status word, grid barrier)
@@ -61,6 +61,13 @@ struct AttnPlan {
 };
 AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs);
 
+// The argument checks of nvfp4kv_quantize_chunk, in its order (need_ws: the
+// workspace pointer is checked too); the no-allocation entry point runs the
+// same checks without a workspace.
+nvfp4kv_status check_quantize_chunk_args(const void* K, const void* V, int T_c, int H, int d,
+                                         const nvfp4kv_chunk_view* out, const void* ws,
+                                         bool need_ws);
+
 nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
                                const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream);
 
@@ -92,21 +99,12 @@ nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, voi
 nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,
                                     cudaStream_t stream);
 
-nvfp4kv_status launch_attention_mma(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
-                                    int H, const void* Q, int T_q, void* O, int o_dtype,
-                                    float softmax_scale, cudaStream_t stream);
-
-nvfp4kv_status launch_attention_tc(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
-                                   int H, const void* Q, int T_q, void* O, int o_dtype,
-                                   float softmax_scale, void* ws, cudaStream_t stream);
-
 nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                    int H, const void* Q, int T_q, void* O, int o_dtype,
                                    float softmax_scale, void* ws, cudaStream_t stream);
 
-// Sink-window attention: the warp-specialized tcgen05 kernel; the environment
-// variable NVFP4KV_ATTENTION_KERNEL selects the single-group tcgen05 kernel
-// ("tc1") or the mma.sync kernel ("mma") instead, for cross-checks.
+// Sink-window attention: the warp-specialized tcgen05 kernel (and its merge
+// kernel for split query blocks).
 nvfp4kv_status launch_attention(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                 int H, const void* Q, int T_q, void* O, int o_dtype,
                                 float softmax_scale, void* ws, cudaStream_t stream);

@@ -530,6 +530,9 @@ __global__ void check_formats_kernel(int op, const float* fin, const uint8_t* bi
             fout[i] = div_markstein(x, D, __frcp_rn(D));
             break;
         }
+        case 5:
+            fout[i] = ex2_poly2(make_float2(fin[i], fin[i])).x;
+            break;
         default:
             break;
     }
@@ -706,27 +709,14 @@ extern "C" nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const vo
                                                          const nvfp4kv_chunk_view* out,
                                                          nvfp4kv_stream_t stream) {
     using namespace nvfp4kv;
-    if (!K || !V || !out || T_c <= 0 || H <= 0 || T_c > (1 << 24) || H > 4096 ||
-        !out->k_codes || !out->k_scales || !out->v_codes || !out->v_scales || !out->k_mean ||
-        !out->tensor_scales)
-        return NVFP4KV_ERR_INVALID_ARG;
-    if (d != kHeadDim) return NVFP4KV_ERR_UNSUPPORTED;
-    const uintptr_t mis = reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) |
-                          reinterpret_cast<uintptr_t>(out->k_codes) |
-                          reinterpret_cast<uintptr_t>(out->v_codes) |
-                          reinterpret_cast<uintptr_t>(out->k_scales) |
-                          reinterpret_cast<uintptr_t>(out->v_scales) |
-                          reinterpret_cast<uintptr_t>(out->k_mean);
-    if ((mis & 15u) != 0 || (reinterpret_cast<uintptr_t>(out->tensor_scales) & 7u) != 0)
-        return NVFP4KV_ERR_ALIGNMENT;
+    // the workspace entry point's checks, in its order
+    const nvfp4kv_status st = check_quantize_chunk_args(K, V, T_c, H, d, out, nullptr, false);
+    if (st != NVFP4KV_OK) return st;
     // the chunk's scratch must fit the compiled-in array
     if (ws_layout(T_c, H).quant_total > kStaticScratchBytes) return NVFP4KV_ERR_CAPACITY;
 
-    int dev = 0, major = 0;
+    int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4KV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-        return NVFP4KV_ERR_CUDA;
-    if (major != 10) return NVFP4KV_ERR_UNSUPPORTED;
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_scratch_mutex);
@@ -740,7 +730,14 @@ extern "C" nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const vo
     }
     // the grid barrier and the status word must start at zero; the partial
     // sums and maxima are written before they are read
-    if (cudaMemsetAsync(scratch, 0, sizeof(Control), (cudaStream_t)stream) != cudaSuccess)
-        return NVFP4KV_ERR_CUDA;
-    return launch_quantize(K, V, T_c, H, *out, scratch, (cudaStream_t)stream);
+    nvfp4kv_status r = NVFP4KV_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, sizeof(Control), (cudaStream_t)stream) == cudaSuccess)
+        r = launch_quantize(K, V, T_c, H, *out, scratch, (cudaStream_t)stream);
+    if (r == NVFP4KV_ERR_CUDA) {
+        // the cached address may be stale (a context that was reset and
+        // recreated reloads the module): look it up again on the next call
+        std::lock_guard<std::mutex> lock(g_scratch_mutex);
+        g_scratch_addr[dev] = nullptr;
+    }
+    return r;
 }

@@ -53,3 +53,53 @@ def sample_rows(T: int, n_random: int = 48, seed: int = 0):
             rows |= {e - 1, e}
     rows |= set(rng.integers(0, T, n_random).tolist())
     return sorted(r for r in rows if 0 <= r < T)
+
+
+# ------------------------------------------------------------------ output canaries
+
+SENTINEL = 0xA5
+GUARD_BYTES = 4096
+
+
+class Guarded:
+    """A device tensor of `shape` and `dtype` with GUARD_BYTES of sentinel bytes
+    right before and after it (its own bytes start as the sentinel too)."""
+
+    def __init__(self, shape, dtype):
+        import torch
+        self.nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.big = torch.full((2 * GUARD_BYTES + self.nbytes,), SENTINEL, dtype=torch.uint8,
+                              device="cuda")
+        self.t = self.big[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype).view(shape)
+
+    def assert_intact(self, what=""):
+        b = self.big.cpu().numpy()
+        head, tail = b[:GUARD_BYTES], b[GUARD_BYTES + self.nbytes:]
+        assert (head == SENTINEL).all() and (tail == SENTINEL).all(), \
+            f"{what}: a store landed outside the output " \
+            f"(guard bytes changed before: {int((head != SENTINEL).sum())}, " \
+            f"after: {int((tail != SENTINEL).sum())})"
+
+
+class GuardedChunk:
+    """A ChunkBuffer carved from a sentinel-filled buffer with GUARD_BYTES on
+    either side; every byte outside the six parts' exact extents (the guards
+    and the alignment padding between parts) must stay the sentinel."""
+
+    def __init__(self, lib, T, H):
+        import torch
+        n = lib.chunk_bytes(T, H)
+        self.big = torch.full((2 * GUARD_BYTES + n + 256,), SENTINEL, dtype=torch.uint8,
+                              device="cuda")
+        self.chunk = lib.ChunkBuffer(T, H, buf=self.big[GUARD_BYTES:GUARD_BYTES + n + 256])
+
+    def assert_intact(self, what=""):
+        c = self.chunk
+        mask = np.ones(self.big.numel(), bool)
+        b0 = self.big.data_ptr()
+        for t in (c.k_codes, c.v_codes, c.k_scales, c.v_scales, c.k_mean, c.tensor_scales):
+            a = t.data_ptr() - b0
+            mask[a:a + t.numel() * t.element_size()] = False
+        rest = self.big.cpu().numpy()[mask]
+        bad = int((rest != SENTINEL).sum())
+        assert bad == 0, f"{what}: {bad} bytes outside the chunk's parts changed"

@@ -195,3 +195,36 @@ def test_binding_fails_loudly_without_library(tmp_path):
             "try:\n    s.load()\nexcept ImportError as e:\n    print('LOUD', e)\n")
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT)
     assert "LOUD" in r.stdout
+
+
+def test_noalloc_refuses_every_bad_argument_as_the_workspace_entry_point(L):
+    """nvfp4kv_quantize_chunk_noalloc runs nvfp4kv_quantize_chunk's argument
+    checks in its order: each bad argument gets the same status from both
+    (nothing reaches the device)."""
+    good = swv.chunk_view_init(FAKE, 64, 2)
+
+    def view(**kw):
+        v = swv.ChunkView(good.k_codes, good.k_scales, good.v_codes, good.v_scales,
+                          good.k_mean, good.tensor_scales)
+        for k, x in kw.items():
+            setattr(v, k, x)
+        return v
+
+    K = V = FAKE + (1 << 24)
+    cases = [
+        dict(K=0), dict(V=0), dict(out=None),
+        dict(T=0), dict(H=0), dict(d=0), dict(d=24), dict(d=64), dict(T=(1 << 24) + 1),
+        dict(H=4097), dict(K=K + 8), dict(V=V + 2),
+        dict(out=view(k_codes=good.k_codes + 8)), dict(out=view(v_scales=good.v_scales + 4)),
+        dict(out=view(k_mean=0)), dict(out=view(tensor_scales=good.tensor_scales + 4)),
+        dict(d=64, K=K + 8), dict(d=24, K=0),
+    ]
+    for c in cases:
+        a = dict(K=K, V=V, T=64, H=2, d=128, out=good)
+        a.update(c)
+        out = ctypes.byref(a["out"]) if a["out"] is not None else None
+        ws_status = L.nvfp4kv_quantize_chunk(a["K"], a["V"], a["T"], a["H"], a["d"], out,
+                                             FAKE, None)
+        na_status = L.nvfp4kv_quantize_chunk_noalloc(a["K"], a["V"], a["T"], a["H"], a["d"],
+                                                     out, None)
+        assert ws_status != swv.OK and na_status == ws_status, (c, ws_status, na_status)

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 import synth
-from gpu_util import assert_attention_close, dev_bf16, host_bf16_to_f64, sample_rows
+from gpu_util import Guarded, assert_attention_close, dev_bf16, host_bf16_to_f64, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -75,7 +75,9 @@ def test_ragged_shapes(lib, orc, T_c, T_q, H):
     import torch
     n_chunks = 3
     chunks, qs = [], []
-    ws = lib.new_workspace(T_c, H)
+    gws = Guarded((lib.workspace_bytes(T_c, H),), torch.uint8)
+    ws = gws.t
+    lib.workspace_init(ws)
     for i in range(n_chunks):
         K = synth.k_with_offsets_bf16(50 + i, T_c, H, (T_c, H, 128))
         V = synth.gaussian_bf16(50 + i, T_c, H, synth.T_V, (T_c, H, 128))
@@ -86,10 +88,13 @@ def test_ragged_shapes(lib, orc, T_c, T_q, H):
     Q = synth.gaussian_bf16(60, T_c, H, synth.T_Q, (T_q, H, 128))
     ref = orc.attention_f64(qs, Q)
     for dt in (torch.float32, torch.bfloat16):
-        O = torch.empty((T_q, H, 128), dtype=dt, device="cuda")
-        lib.attention(chunks, dev_bf16(Q), O, ws)
+        gO = Guarded((T_q, H, 128), dt)
+        lib.attention(chunks, dev_bf16(Q), gO.t, ws)
         torch.cuda.synchronize()
-        assert_attention_close(host_bf16_to_f64(O), ref, f"T_c={T_c} T_q={T_q} {dt}",
+        assert lib.workspace_status(ws) == lib.OK
+        gO.assert_intact(f"O T_c={T_c} T_q={T_q} {dt}")
+        gws.assert_intact(f"workspace T_c={T_c} T_q={T_q} {dt}")
+        assert_attention_close(host_bf16_to_f64(gO.t), ref, f"T_c={T_c} T_q={T_q} {dt}",
                                bf16_output=dt == torch.bfloat16)
 
 

@@ -78,3 +78,26 @@ def test_quotient_is_correctly_rounded(lib, orc):
     want = (x / D).astype(np.float32)
     bad = np.nonzero(got.view(np.uint32) != want.view(np.uint32))[0]
     assert bad.size == 0, f"{bad.size} quotients differ, e.g. x={x[bad[:4]]} D={D[bad[:4]]}"
+
+
+def test_softmax_ex2_polynomial_within_its_bound(lib):
+    """The attention softmax's 2^x on the FMA pipe (Cody-Waite style split into
+    n + f, a least-squares cubic for 2^f on [-1/2, 1/2]): relative error at most
+    7.6e-5 (7.504e-5 for the cubic itself, plus fp32 rounding) against exp2 in
+    float64, over its input range [-126, 8] -- every integer and half-integer
+    point, their fp32 neighbours, and a dense random sweep."""
+    import torch
+    rng = np.random.default_rng(31)
+    grid = np.arange(-252, 17, dtype=np.float64) / 2.0            # n and n + 1/2
+    g32 = grid.astype(np.float32)
+    pts = np.concatenate([g32, np.nextafter(g32, np.float32(-np.inf)),
+                          np.nextafter(g32, np.float32(np.inf))])
+    x = np.concatenate([pts, rng.uniform(-126.0, 8.0, 4_000_000).astype(np.float32),
+                        rng.uniform(-1.0, 1.0, 1_000_000).astype(np.float32)])
+    x = np.clip(x, np.float32(-126.0), np.float32(8.0)).astype(np.float32)
+    got = _run(lib, 5, x, torch.float32).astype(np.float64)
+    want = np.exp2(x.astype(np.float64))
+    rel = np.abs(got / want - 1.0)
+    worst = int(np.argmax(rel))
+    assert rel[worst] <= 7.6e-5, f"x={x[worst]!r}: 2^x {want[worst]!r}, got {got[worst]!r}"
+    assert rel.mean() < 5e-5

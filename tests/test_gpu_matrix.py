@@ -22,14 +22,26 @@ def _matrix(seed, M, N, outlier=30.0):
     return synth.to_bf16_bits(np.where(u < 0.01, z * outlier, z))
 
 
-def _check(lib, orc, X, mode, ws=None, what=""):
+def _check(lib, orc, X, mode, ws=None, what="", guard=False):
+    """Quantize on the GPU and compare with the oracle; with guard, every
+    output sits between sentinel guards that must stay untouched."""
     import torch
+    from gpu_util import Guarded
     M, N = X.shape
     ws = lib.new_matrix_workspace() if ws is None else ws
     out = lib.MatrixBuffer(M, N, mode)
+    guards = []
+    if guard:
+        for name in ("codes", "scales", "tensor_scale"):
+            t = getattr(out, name)
+            g = Guarded(tuple(t.shape), t.dtype)
+            setattr(out, name, g.t)
+            guards.append((name, g))
     lib.quantize_matrix(_dev(X), out, ws)
     torch.cuda.synchronize()
     assert lib.workspace_status(ws) == lib.OK
+    for name, g in guards:
+        g.assert_intact(f"{what} {name}")
     got, ref = out.to_host(), orc.quantize_matrix(X, mode)
     assert np.float32(got["s"]) == np.float32(ref["s"]), f"{what} tensor scale"
     for k in ("scales", "codes"):
@@ -48,7 +60,7 @@ def test_dit_shapes_bit_exact(lib, orc, mode, M, N):
 @pytest.mark.parametrize("mode,M,N", [(1, 1, 16), (1, 7, 48), (1, 33, 272), (1, 130, 528),
                                       (2, 16, 16), (2, 48, 80), (2, 160, 304)])
 def test_ragged_shapes_bit_exact(lib, orc, mode, M, N):
-    _check(lib, orc, _matrix(7 + M + N, M, N), mode, what=f"{M}x{N}")
+    _check(lib, orc, _matrix(7 + M + N, M, N), mode, what=f"{M}x{N}", guard=True)
 
 
 @pytest.mark.parametrize("mode", [1, 2])

@@ -6,19 +6,24 @@ import numpy as np
 import pytest
 
 import synth
-from gpu_util import dev_bf16
+from gpu_util import Guarded, GuardedChunk, dev_bf16
 
 pytestmark = pytest.mark.gpu
 
 
-def _gpu_quant(lib, K, V, ws=None):
+def _gpu_quant(lib, K, V, ws=None, guard=False):
+    """Quantize on the GPU; with guard, into a chunk carved from a sentinel
+    buffer whose bytes outside the chunk's parts are checked afterwards."""
     import torch
     T, H, d = K.shape
     ws = lib.new_workspace(T, H, d) if ws is None else ws
-    out = lib.ChunkBuffer(T, H, d)
+    g = GuardedChunk(lib, T, H) if guard else None
+    out = g.chunk if guard else lib.ChunkBuffer(T, H, d)
     lib.quantize_chunk(dev_bf16(K), dev_bf16(V), out, ws)
     torch.cuda.synchronize()
     assert lib.workspace_status(ws) == lib.OK
+    if guard:
+        g.assert_intact(f"quantize T={T} H={H}")
     return out, ws
 
 
@@ -53,7 +58,7 @@ def test_quantize_only_full_size_bit_exact(lib, orc, index):
 def test_ragged_shapes_bit_exact(lib, orc, T, H):
     K = synth.k_with_offsets_bf16(31, T, H, (T, H, 128), outlier_mult=50.0)
     V = synth.gaussian_bf16(31, T, H, synth.T_V, (T, H, 128))
-    out, _ = _gpu_quant(lib, K, V)
+    out, _ = _gpu_quant(lib, K, V, guard=True)
     _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"T={T} H={H}")
 
 
@@ -146,14 +151,16 @@ def test_dequantize_ragged_tiles_bit_exact(lib, orc, T, H, bf16_out):
     import torch
     K = synth.k_with_offsets_bf16(57, T, H, (T, H, 128), outlier_mult=20.0)
     V = synth.gaussian_bf16(57, T, H, synth.T_V, (T, H, 128))
-    out, _ = _gpu_quant(lib, K, V)
+    out, _ = _gpu_quant(lib, K, V, guard=True)
     q = orc.quantize_chunk(K, V)
     _assert_same(out.to_host(), q, f"T={T} H={H}")
     dt = torch.bfloat16 if bf16_out else torch.float32
-    Kd = torch.empty((T, H, 128), dtype=dt, device="cuda")
-    Vd = torch.empty((T, H, 128), dtype=dt, device="cuda")
+    gK, gV = Guarded((T, H, 128), dt), Guarded((T, H, 128), dt)
+    Kd, Vd = gK.t, gV.t
     lib.dequantize(out, Kd, Vd)
     torch.cuda.synchronize()
+    gK.assert_intact(f"de-quantized K T={T} H={H}")
+    gV.assert_intact(f"de-quantized V T={T} H={H}")
     Kr = orc.dequantize_tensor(q["k_codes"], q["k_scales"], q["k_mean"], q["s_k"], T, H, 128)
     Vr = orc.dequantize_tensor(q["v_codes"], q["v_scales"], None, q["s_v"], T, H, 128)
     for name, got, want in (("K", Kd, Kr), ("V", Vd, Vr)):

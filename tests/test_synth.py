@@ -33,3 +33,27 @@ def test_recipe_moments():
     dev = Kq - Kq.mean(axis=0, keepdims=True)
     frac_big = (np.abs(dev) > 8).mean()           # outliers x20 on 1% of elements
     assert 0.005 < frac_big < 0.012
+
+
+def test_device_generator_matches_the_host_one():
+    """synth.device (torch, here on the CPU) draws the same bits as the host
+    generator: words, uniforms, and the bf16 recipes of the quantize-only chunk."""
+    import torch
+
+    import synth.device as sd
+    key = synth.stream_key(7, 1, 2, synth.T_K)
+    assert np.array_equal(sd.words(key, 1000, "cpu").numpy().view(np.uint64),
+                          synth.words(key, 1000))
+    assert np.array_equal(sd.uniform(key, 999, "cpu").numpy(), synth.uniform(key, 999))
+    shape = (96, 3, 128)
+    K = sd.k_with_offsets_bf16(5, 0, 0, shape, "cpu")
+    V = sd.gaussian_bf16(5, 0, 0, synth.T_V, shape, "cpu")
+    assert K.dtype == torch.bfloat16 and tuple(K.shape) == shape
+    assert np.array_equal(K.view(torch.int16).numpy().view(np.uint16),
+                          synth.k_with_offsets_bf16(5, 0, 0, shape))
+    assert np.array_equal(V.view(torch.int16).numpy().view(np.uint16),
+                          synth.gaussian_bf16(5, 0, 0, synth.T_V, shape))
+    Kq, Vq = sd.quant_chunk(3, "cpu", T_c=64, H=2)
+    Kh, Vh = synth.quant_chunk(3, T_c=64, H=2)
+    assert np.array_equal(Kq.view(torch.int16).numpy().view(np.uint16), Kh)
+    assert np.array_equal(Vq.view(torch.int16).numpy().view(np.uint16), Vh)

@@ -49,15 +49,39 @@ def test_noalloc_matches_workspace_entry_point_twice(lib):
             assert np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)), f"call {call}: {k}"
 
 
+def test_noalloc_at_its_largest_chunk(lib):
+    """T_c = 10,816 at H = 24 fills the compiled-in scratch to within 8 KB of its
+    end: the same bytes as the workspace entry point, twice in a row."""
+    import torch
+    T, H, d = 10816, 24, 128
+    K = synth.k_with_offsets_bf16(91, 0, 0, (T, H, d))
+    V = synth.gaussian_bf16(91, 0, 0, synth.T_V, (T, H, d))
+    Kd, Vd = dev_bf16(K), dev_bf16(V)
+    ref = lib.ChunkBuffer(T, H, d)
+    ws = lib.new_workspace(T, H, d)
+    lib.quantize_chunk(Kd, Vd, ref, ws)
+    b = _parts(ref)
+    for call in range(2):
+        got = lib.ChunkBuffer(T, H, d)
+        lib.quantize_chunk_noalloc(Kd, Vd, got)
+        torch.cuda.synchronize()
+        a = _parts(got)
+        for k in a:
+            assert np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)), f"call {call}: {k}"
+    assert lib.workspace_status(ws) == lib.OK
+
+
 def test_noalloc_refuses_chunks_beyond_its_scratch(lib):
     import torch
     fn = _entry(lib)
     K = torch.zeros((16, 2, 128), dtype=torch.bfloat16, device="cuda")
     buf = lib.ChunkBuffer(16, 2)
-    # 10,880 tokens x 24 heads needs more than the 4 MiB compiled-in scratch;
-    # refused from the sizes alone, before anything reads K
-    st = fn(K.data_ptr(), K.data_ptr(), 10880, 24, 128, ctypes.byref(buf.view),
-            torch.cuda.current_stream().cuda_stream)
-    assert st == lib.ERR_CAPACITY
+    # one token past the largest chunk (10,817 x 24 needs a 170th 64-token
+    # segment: more than the 4 MiB compiled-in scratch); refused from the sizes
+    # alone, before anything reads K
+    for T in (10817, 10880):
+        st = fn(K.data_ptr(), K.data_ptr(), T, 24, 128, ctypes.byref(buf.view),
+                torch.cuda.current_stream().cuda_stream)
+        assert st == lib.ERR_CAPACITY
     assert fn(K.data_ptr(), K.data_ptr(), 16, 2, 64, ctypes.byref(buf.view), None) \
         == lib.ERR_UNSUPPORTED
