@@ -112,8 +112,11 @@ size_t nvfp4kv_workspace_bytes(int T_c, int H, int d);
  * NVFP4KV_ERR_DEVICE_TIMEOUT. */
 nvfp4kv_status nvfp4kv_workspace_init(void* ws, size_t ws_bytes, nvfp4kv_stream_t stream);
 
-/* Synchronize `stream`, read the workspace's status word (OK or
- * NVFP4KV_ERR_DEVICE_TIMEOUT) and clear it. */
+/* Synchronize `stream`, read the workspace's status word and clear it:
+ * NVFP4KV_OK, NVFP4KV_ERR_DEVICE_TIMEOUT (a bounded wait inside a kernel gave
+ * up), or NVFP4KV_ERR_UNSUPPORTED (an attention call met a key set whose V
+ * tensor scales span more than 2^116, beyond what its fp32 softmax sums hold;
+ * that call's output is not valid).  A timeout outranks the other. */
 nvfp4kv_status nvfp4kv_workspace_status(void* ws, nvfp4kv_stream_t stream);
 
 /* ------------------------------------------------------------------ quantizer */
@@ -315,9 +318,12 @@ nvfp4kv_status nvfp4kv_dequantize(const nvfp4kv_chunk_view* in, int T_c, int H, 
  *           NVFP4KV_BF16).
  *   softmax_scale: <= 0 selects 1/sqrt(d).
  *   ws:     workspace as for the quantizer (status word only).
- * Softmax statistics are fp32; the products run on the tensor cores in bf16
- * with the de-quantized values exact in bf16; the normalized result is
- * stored in o_dtype.
+ * Softmax statistics are fp32; the products run on the tensor cores in fp16
+ * (the de-quantized codes times their block scales are exact fp16 numbers;
+ * Q is scaled by a power of two into fp16 range; s_K, the K mean and s_V
+ * enter in fp32); the normalized result is stored in o_dtype.  Chunks' V
+ * tensor scales may differ by up to 2^116 within one key set; a wider spread
+ * is reported by nvfp4kv_workspace_status as NVFP4KV_ERR_UNSUPPORTED.
  */
 nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
                                  int T_c, int H, int d, const void* Q, int T_q,
@@ -427,7 +433,8 @@ nvfp4kv_status kvcache_check_status(kvcache* cache, nvfp4kv_stream_t stream);
  * op 1: E4M3 byte of each fp32 input, op 2: fp32 value of each E2M1 code,
  * op 3: fp32 value of each E4M3 byte, op 4: the fp32 quotient x/D that the
  * quantizer forms for a pair (in[2i] = x, in[2i+1] = D > 0), op 5: 2^x
- * by the attention softmax's polynomial on the FMA pipe (for x >= -126).
+ * by the attention softmax's polynomial on the FMA pipe (inputs below -125
+ * are taken as -125).
  * in/out are device arrays of n elements (op 4: n quotients from 2n inputs).
  */
 nvfp4kv_status nvfp4kv_check_formats(int op, const void* in, void* out, size_t n,

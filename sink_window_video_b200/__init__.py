@@ -275,7 +275,9 @@ def workspace_init(ws, stream=None):
 
 
 def workspace_status(ws, stream=None) -> int:
-    """Synchronize and return the workspace status code (OK or ERR_DEVICE_TIMEOUT)."""
+    """Synchronize and return the workspace status code and clear it: OK,
+    ERR_DEVICE_TIMEOUT (a bounded wait in a kernel gave up) or ERR_UNSUPPORTED
+    (an attention key set whose V tensor scales span more than 2^116)."""
     return int(load().nvfp4kv_workspace_status(_ptr(ws), _stream(stream)))
 
 

@@ -192,7 +192,8 @@ nvfp4kv_status nvfp4kv_workspace_status(void* ws, nvfp4kv_stream_t stream) {
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return NVFP4KV_ERR_CUDA;
-    return NVFP4KV_ERR_DEVICE_TIMEOUT;
+    // a wait that gave up outranks an input the attention could not represent
+    return (st & 1u) ? NVFP4KV_ERR_DEVICE_TIMEOUT : NVFP4KV_ERR_UNSUPPORTED;
 }
 
 nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int H, int d,

@@ -9,15 +9,16 @@
 // tensor-core operands, s_K and the K-smoothing bias Q.mean_c enter the fp32
 // logits, s_V/s_Vmax scales P per chunk, and Q rows are scaled by powers of two
 // into fp16 range.
-// Two running references per row (log2 units), because the chunks' V scales
-// may differ by many binades:
-//   m_o  for P' = 2^(x + v_c - m_o), v_c = log2(s_V,c / s_Vmax): P' measures a
-//        key's contribution to O, so the keys that carry O are normal fp16
-//        numbers whichever chunk they come from;
-//   m_l  for the fp32 row sum l = sum 2^(x - m_l) of the softmax denominator,
-//        taken per tile as sum(P') 2^(m_o - v_c - m_l), or, for a chunk whose
-//        V scale is below 2^-48 of the largest, from its own exponentials.
-// O = O_acc 2^(m_o + log2 s_Vmax - m_l) / l.
+// The chunks' V scales may differ by many binades, so the running reference
+// m of each row (log2 units) is the maximum of x + v_c, the logit plus
+// v_c = log2(s_V,c / s_Vmax): P' = 2^(x + v_c - m) measures a key's share of
+// O, and the keys that carry O are normal fp16 numbers whichever chunk they
+// come from (v_c is folded into the chunk's logit bias).  The fp32 row sum
+// l = sum 2^(x - m) is taken per tile as sum(P') 2^(-v_c), or, for a chunk
+// whose V scale is below 2^-48 of the largest (its P' may underflow while its
+// keys still weigh in the denominator), from the keys' own exponentials.  A
+// key set whose V scales span more than 2^116 would overflow that sum; the
+// kernel reports it (kStatusRange) instead.
 //
 // One CTA per SM: a head and 256 query rows (two 128-row tiles Q0, Q1), keys
 // in 128-key tiles.  Warp roles (384 threads; 12 warps keep 168 registers per
@@ -72,8 +73,10 @@ constexpr size_t kSmemW = (2 + 2 * kStages) * kTileB + 1024;
 constexpr float kLog2eW = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 // A chunk whose V tensor scale is below 2^-kFarLog2 of the key set's largest
-// takes its softmax denominator from its own exponentials (see above).
+// takes its softmax denominator from its own exponentials (see above); below
+// 2^-kRangeLog2 the denominator could overflow and the call is reported.
 constexpr float kFarLog2 = 48.0f;
+constexpr float kRangeLog2 = 116.0f;
 
 struct WsChunk {
     const uint8_t* k_codes;
@@ -272,16 +275,16 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         auto log2_svmax = [&]() {
             float v = 0.0f;
             for (int ci = 0; ci < a.n_chunks; ++ci) v = fmaxf(v, a.chunk[ci].tensor_scales[1]);
-            return __log2f(v);
+            return log2f(v);
         };
 
-        float m_o = -INFINITY, m_l = -INFINITY, l_run = 0.0f;
+        float m_run = -INFINITY, l_run = 0.0f;
         bool o_written = false, ok = true;
         int t = 0;
         const uint32_t s_full = smem_u32(&sh.s_full[qi]);
         const uint32_t p_full = smem_u32(&sh.p_full[qi]);
         int ci_cur = -1;
-        float alpha = 0.0f, beta = 0.0f, lrV = 0.0f;
+        float alpha = 0.0f, beta = 0.0f, lrV = 0.0f, inv_rV = 0.0f;
         float2 alpha2 = make_float2(0.0f, 0.0f);
         for (; t < ntiles && ok; ++t) {
             const int gt = t_begin + t;                        // global tile index
@@ -306,9 +309,14 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                     }
                 }
                 alpha = qexp * sK * a.scale_log2;
-                beta = qmu * a.scale_log2;
-                lrV = __log2f(sV) - log2_svmax();
+                // (log2f: exact enough and defined for subnormal scales; clamped
+                // so that a reported out-of-range key set stays finite)
+                lrV = fmaxf(log2f(sV) - log2_svmax(), -126.0f);
+                beta = fmaf(qmu, a.scale_log2, lrV);           // logit bias + v_c
+                inv_rV = ex2f(-lrV);
                 alpha2 = make_float2(alpha, alpha);
+                if (lrV < -kRangeLog2 && r == 0 && (warp & 3) == 0)
+                    atomicOr(&a.ctl->status, kStatusRange);
             }
             {
                 bool got = wait_or_abort(s_full, (uint32_t)(t & 1), abort, a.ctl, 10u + qi, t);
@@ -345,19 +353,13 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                                      fmaxf(m8[6], m8[7]));
                     mx = fmaf(mx, alpha, beta);                 // alpha > 0: same argmax
                     // (a half without valid keys has mx = -inf and never grows)
-                    const float mv = mx + lrV;
-                    if (mx > m_l + kRescaleLog2 || (m_l == -INFINITY && mx > -INFINITY)) {
-                        const float m_new = fmaxf(mx, m_l);
-                        const float cl = ex2f(m_l - m_new);
-                        l_run *= cl;
-                        m_l = m_new;
-                    }
-                    const bool grow = mv > m_o + kRescaleLog2 || (m_o == -INFINITY && mv > -INFINITY);
+                    const bool grow = mx > m_run + kRescaleLog2 || (m_run == -INFINITY && mx > -INFINITY);
                     float corr = 1.0f;
                     if (grow) {
-                        const float m_new = fmaxf(mv, m_o);
-                        corr = ex2f(m_o - m_new);
-                        m_o = m_new;
+                        const float m_new = fmaxf(mx, m_run);
+                        corr = ex2f(m_run - m_new);
+                        l_run *= corr;
+                        m_run = m_new;
                     }
                     if (__any_sync(0xFFFFFFFFu, grow)) {
                         // rare: rescale what this row holds with the old max --
@@ -393,10 +395,27 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                             }
                         }
                     }
-                    // p' = 2^(logit + log2(s_V/s_Vmax) - m_o), one fused multiply-add
+                    if (lrV < -kFarLog2) {
+                        // (rare, chunk-uniform) the tile's P' may underflow while
+                        // its keys still weigh in the denominator: 2^(x - m),
+                        // from S re-read in tensor memory (small code)
+                        const float bl = beta - lrV - m_run;
+                        float al = 0.0f;
+#pragma unroll 1
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t sv[16];
+                            tmem_ld16(tS + 64 * hh + 16 * q, sv);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int k = 0; k < 16; ++k)
+                                if (16 * q + k < vh) al += ex2f(fmaf(__uint_as_float(sv[k]), alpha, bl));
+                        }
+                        l_run += al;
+                    }
+                    // p' = 2^(logit + log2(s_V/s_Vmax) - m), one fused multiply-add
                     // each; two of every eight pairs on the FMA pipe, the rest on
                     // the special-function unit; four independent partial sums
-                    const float b2 = beta - m_o + lrV;
+                    const float b2 = beta - m_run;
                     const float2 b22 = make_float2(b2, b2);
                     uint32_t p[32];
 #pragma unroll
@@ -414,22 +433,12 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                     }
                     __syncwarp();
                     tmem_st32(tS + 32 * hh, p);
-                    if (lrV < -kFarLog2) {
-                        // (rare, chunk-uniform) the tile's P' may underflow while
-                        // its keys still weigh in the denominator: 2^(x - m_l)
-                        const float bl = beta - m_l;
-                        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                        for (int k = 0; k < 64; ++k)
-                            a4[k & 3] += ex2f(fmaf(__uint_as_float(s[k]), alpha, bl));
-                        l_run += (a4[0] + a4[1]) + (a4[2] + a4[3]);
-                    }
                 }
                 tmem_wait_st();
                 if (!(lrV < -kFarLog2)) {
                     const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
                     const float2 a03 = __fadd2_rn(a01, a23);
-                    l_run += (a03.x + a03.y) * ex2f(m_o - lrV - m_l);
+                    l_run += (a03.x + a03.y) * inv_rV;
                 }
                 tc_fence_before();
                 mbar_arrive(p_full);
@@ -442,8 +451,9 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
         }
         if (ok) {
             tc_fence_after();
-            const float lsVmax = log2_svmax();
-            const float inv = ex2f(m_o + lsVmax - m_l) / l_run;
+            float sVmax = 0.0f;
+            for (int ci = 0; ci < a.n_chunks; ++ci) sVmax = fmaxf(sVmax, a.chunk[ci].tensor_scales[1]);
+            const float inv = sVmax / l_run;
             // a split block leaves its unnormalized O, running max and row sum
             // (in units where O / l is the output) for the merge kernel
             float* prow = split ? a.part + ((size_t)piece * 256 + qi * 128 + r) * kPartialFloats
@@ -485,9 +495,8 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
                 }
             }
             if (rvalid && split) {
-                prow[128] = m_o + lsVmax;
-                prow[129] = m_l;
-                prow[130] = l_run;
+                prow[128] = m_run;
+                prow[129] = l_run / sVmax;
             }
         }
     } else if (warp >= kDequantWarp0) {
@@ -633,11 +642,9 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
     }
 }
 
-// Merge of a split query block: per row, over its key ranges q (each with its
-// unnormalized O_q in units of 2^(mo_q), its row sum l_q in units of
-// 2^(ml_q)): Mo = max mo_q, Ml = max ml_q,
-// O = sum 2^(mo_q - Mo) O_q 2^(Mo - Ml) / sum 2^(ml_q - Ml) l_q.
-// One warp per row, four outputs per lane.
+// Merge of a split query block: per row, M = max m_q, O = sum 2^(m_q - M) O_q /
+// sum 2^(m_q - M) l_q over its key ranges q.  One warp per row, four outputs
+// per lane.
 __global__ void __launch_bounds__(256) attention_merge_kernel(const float* part, int n_full,
                                                               int n_tail, int n_split,
                                                               int pairs_per_head, int T_q, int H,
@@ -652,24 +659,21 @@ __global__ void __launch_bounds__(256) attention_merge_kernel(const float* part,
     if (row >= T_q) return;
     const float* base = part + ((size_t)tp * n_split * 256 + rr) * kPartialFloats;
     const size_t stride = (size_t)256 * kPartialFloats;
-    float Mo = -INFINITY, Ml = -INFINITY;
-    for (int q = 0; q < n_split; ++q) {
-        Mo = fmaxf(Mo, base[q * stride + 128]);
-        Ml = fmaxf(Ml, base[q * stride + 129]);
-    }
+    float M = -INFINITY;
+    for (int q = 0; q < n_split; ++q) M = fmaxf(M, base[q * stride + 128]);
     float L = 0.0f;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int q = 0; q < n_split; ++q) {
         const float* pq = base + q * stride;
-        const float wq = exp2f(pq[128] - Mo);
-        L = fmaf(exp2f(pq[129] - Ml), pq[130], L);
+        const float wq = exp2f(pq[128] - M);
+        L = fmaf(wq, pq[129], L);
         const float4 o = reinterpret_cast<const float4*>(pq)[lane];
         acc.x = fmaf(wq, o.x, acc.x);
         acc.y = fmaf(wq, o.y, acc.y);
         acc.z = fmaf(wq, o.z, acc.z);
         acc.w = fmaf(wq, o.w, acc.w);
     }
-    const float inv = exp2f(Mo - Ml) / L;
+    const float inv = 1.0f / L;
     const size_t o = ((size_t)row * H + h) * kHeadDim + 4 * lane;
     if (o_f32) {
         *reinterpret_cast<float4*>(static_cast<float*>(O) + o) =

@@ -19,6 +19,7 @@ constexpr float kTensorScaleDiv = 2688.0f;   // 6 * 448
 
 // Status bits recorded by kernels in the workspace.
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusRange = 2u;   // attention: key set's V scales span more than 2^116
 
 // Time limit of any single wait inside a kernel, in nanoseconds; a wait that
 // reaches it records kStatusTimeout (and its site) and the kernel returns.
@@ -193,11 +194,12 @@ __device__ __forceinline__ float div_markstein(float x, float D, float r) {
 // scarcer resource):
 // n = round(x) by adding and subtracting 1.5*2^23, f = x - n in [-1/2, 1/2],
 // 2^f by a cubic (least-squares fit on relative error, max 7.5e-5), and 2^n
-// added to the exponent field.  x is clamped to -126 so 2^n stays normal;
-// inputs here are at most 8 (the lazy-max bound).
+// added to the exponent field.  x is clamped to -125 so the result stays a
+// normal number (2^f may be just below 1); the softmax's inputs are at most 8
+// (the lazy-max bound), and below 2^-125 its values round to zero in fp16.
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -126.0f);
-    x.y = fmaxf(x.y, -126.0f);
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
     const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
     const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
     const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));

@@ -16,11 +16,11 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Attention work split (see launch_attention_ws): the 256-row query blocks
 // that do not fill a whole wave of CTAs are split into up to kMaxSplit key
-// ranges, whose partial results (per row: 128 fp32 outputs, the two running maxima
+// ranges, whose partial results (per row: 128 fp32 outputs, the running max
 // and the row sum) go to the workspace and are merged by a second kernel.
 constexpr int kMaxTailPairs = 160;   // more than one wave never remains
 constexpr int kMaxSplit = 8;
-constexpr int kPartialFloats = 132;  // per row: O[128], m_o, m_l, l, 1 pad (16-byte rows)
+constexpr int kPartialFloats = 132;  // per row: O[128], m, l, 2 pad (16-byte rows)
 
 // Workspace layout for chunks of T tokens and H heads (d = 128):
 //   [0, 256)  Control (status word, grid barrier)

@@ -105,3 +105,28 @@ def test_vscale_spread_whole_blocks(lib, orc, mass, log2r):
     """148 whole query blocks (one full wave, no split): the kernel normalizes
     its rows itself."""
     _run(lib, orc, mass, log2r, T_c=136, H=4, T_q=37 * 256, seed=500 + log2r)
+
+
+def test_vscale_spread_beyond_range_is_reported(lib, orc):
+    """V scales 2^120 apart exceed what the fp32 softmax sums hold: the call is
+    reported as ERR_UNSUPPORTED by the status check (not silently wrong), and
+    the next in-range call on the same workspace is OK and correct."""
+    import torch
+    T_c, H, T_q = 136, 2, 200
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i, (v_log2, k0) in enumerate([(-120.0, 0.0), (0.0, 0.0)]):
+        K, V = _chunk(700 + i, T_c, H, v_log2, k0)
+        b = lib.ChunkBuffer(T_c, H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), b, ws)
+        bufs.append(b)
+        qs.append(orc.quantize_chunk(K, V))
+    Q = synth.gaussian_bf16(709, 0, 0, synth.T_Q, (T_q, H, 128))
+    O = torch.empty((T_q, H, 128), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    lib.attention(bufs, dev_bf16(Q), O, ws)
+    assert lib.workspace_status(ws) == lib.ERR_UNSUPPORTED
+    lib.attention(bufs[1:], dev_bf16(Q), O, ws)
+    assert lib.workspace_status(ws) == lib.OK
+    assert_attention_close(host_to_f64(O), orc.attention_f64(qs[1:], Q), "after the report")

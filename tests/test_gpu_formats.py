@@ -84,20 +84,24 @@ def test_softmax_ex2_polynomial_within_its_bound(lib):
     """The attention softmax's 2^x on the FMA pipe (Cody-Waite style split into
     n + f, a least-squares cubic for 2^f on [-1/2, 1/2]): relative error at most
     7.6e-5 (7.504e-5 for the cubic itself, plus fp32 rounding) against exp2 in
-    float64, over its input range [-126, 8] -- every integer and half-integer
-    point, their fp32 neighbours, and a dense random sweep."""
+    float64, over its input range [-125, 8] -- every integer and half-integer
+    point, their fp32 neighbours, and a dense random sweep -- and inputs below
+    the range are taken as -125."""
     import torch
     rng = np.random.default_rng(31)
-    grid = np.arange(-252, 17, dtype=np.float64) / 2.0            # n and n + 1/2
+    grid = np.arange(-250, 17, dtype=np.float64) / 2.0            # n and n + 1/2
     g32 = grid.astype(np.float32)
     pts = np.concatenate([g32, np.nextafter(g32, np.float32(-np.inf)),
                           np.nextafter(g32, np.float32(np.inf))])
-    x = np.concatenate([pts, rng.uniform(-126.0, 8.0, 4_000_000).astype(np.float32),
+    x = np.concatenate([pts, rng.uniform(-125.0, 8.0, 4_000_000).astype(np.float32),
                         rng.uniform(-1.0, 1.0, 1_000_000).astype(np.float32)])
-    x = np.clip(x, np.float32(-126.0), np.float32(8.0)).astype(np.float32)
+    x = np.clip(x, np.float32(-125.0), np.float32(8.0)).astype(np.float32)
     got = _run(lib, 5, x, torch.float32).astype(np.float64)
     want = np.exp2(x.astype(np.float64))
     rel = np.abs(got / want - 1.0)
     worst = int(np.argmax(rel))
     assert rel[worst] <= 7.6e-5, f"x={x[worst]!r}: 2^x {want[worst]!r}, got {got[worst]!r}"
     assert rel.mean() < 5e-5
+    low = np.float32([-125.5, -126.0, -130.0, -1000.0])
+    assert np.array_equal(_run(lib, 5, low, torch.float32),
+                          _run(lib, 5, np.full(4, -125.0, np.float32), torch.float32))
