@@ -34,7 +34,14 @@ struct Control {
     unsigned test_flags;  // test hooks, 0 in normal use (bit 0: see attention_ws.cu)
     unsigned pad0;
     unsigned long long stamp[8];   // %globaltimer at CTA 0's phase boundaries (diagnostics)
-    unsigned pad[38];
+    // the chunk quantizer's progress across CTAs (its last CTA resets them)
+    unsigned q_vdone;     // CTAs whose max |V| is folded into q_vmax
+    unsigned q_vmax;      // max |V| (float bits: non-negative floats order as their bits)
+    unsigned q_sdone;     // K statistics units written
+    unsigned q_fdone;     // 32-column blocks whose mean is written
+    unsigned q_kmax;      // max |K - mean| (float bits)
+    unsigned q_exit;      // CTAs finished
+    unsigned pad[32];
 };
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {

@@ -170,6 +170,83 @@ __device__ __noinline__ float2 ratio_slow(float ab, float ms6, float ms4) {
     return make_float2(__fdiv_rn(ab, ms6), __fdiv_rn(ab, ms4));
 }
 
+// ---------------------------------------------------------------- Four-Over-Six block encoder
+//
+// The choice between the two candidates needs their squared errors E6, E4 in
+// the definition's fp32 order only when they are close.  Each candidate's
+// error is first estimated with one fused multiply-add per element,
+// e' = RN(x - dq D), squared and summed in pairs; the estimate differs from
+// the definition's sum E by at most 27.3 u S + 4.2 u ab^2 (u = 2^-24, S the
+// exact sum of the real errors, ab the block max; derived from one rounding
+// per product and sum step and |dq D| <= |x| + |e|).  When |E4' - E6'| is
+// above 2^-16 (E4' + E6') + 2^-18 ab^2 -- several times that bound for the
+// two candidates together -- the estimates decide; otherwise both sums are
+// recomputed in the definition's order.  Codes come from the correctly
+// rounded quotients either way, so the result is the definition's, bit for
+// bit.
+
+// Below this block max the estimate's error analysis (no underflow) is not
+// relied on: the exact sums decide.
+constexpr float kApproxMinBlockMax = 0x1p-50f;
+
+// Eight elements against one candidate (D, r = RN(1/D)): the packed codes of
+// -x / D (Markstein's quotient, which keeps the sign of zero) and their
+// decoded values dq' = -sign(x) |dq| as fp32 pairs.
+__device__ __forceinline__ uint32_t quot_codes(const float2* x, float2 Dr, float2* dq) {
+    const float2 NR = make_float2(-Dr.y, -Dr.y);
+    const float2 D2 = make_float2(Dr.x, Dr.x);
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 n0 = __fmul2_rn(x[j], NR);
+        const float2 e = __ffma2_rn(n0, D2, x[j]);
+        const float2 n1 = __ffma2_rn(e, NR, n0);
+        y[2 * j] = n1.x;
+        y[2 * j + 1] = n1.y;
+    }
+    uint32_t h[4];
+    const uint32_t q = cvt_e2m1x8_dec(y, h);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dq[j] = f16x2_to_f32x2(h[j]);
+    return q;
+}
+
+// The estimate of one half block's squared error: sum RN(x + dq' D)^2 in pairs.
+__device__ __forceinline__ float sse_estimate(const float2* x, const float2* dq, float D) {
+    const float2 D2 = make_float2(D, D);
+    float2 e = __ffma2_rn(dq[0], D2, x[0]);
+    float2 acc = __fmul2_rn(e, e);
+#pragma unroll
+    for (int j = 1; j < 4; ++j) {
+        e = __ffma2_rn(dq[j], D2, x[j]);
+        acc = __ffma2_rn(e, e, acc);
+    }
+    return __fadd_rn(acc.x, acc.y);
+}
+
+// The definition's sum for one half block (elements in order): codes q of
+// -x / D, step D.  Out of line: it runs only when the estimates are too close.
+__device__ __noinline__ float sse_exact(float x0, float x1, float x2, float x3, float x4,
+                                        float x5, float x6, float x7, uint32_t q, float D,
+                                        float one) {
+    const float2 x[4] = {make_float2(x0, x1), make_float2(x2, x3), make_float2(x4, x5),
+                         make_float2(x6, x7)};
+    uint32_t h[4];
+    cvt_e2m1x8_to_f16x2(q, h);
+    const float2 D2 = make_float2(D, D);
+    const float2 ONE = make_float2(one, one);
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 p = __fmul2_rn(f16x2_to_f32x2(h[j]), D2);      // RN(dq' D) = -RN(dq D)
+        const float2 d = __ffma2_rn(p, ONE, x[j]);                   // RN(x - RN(dq D))
+        const float2 sq = __fmul2_rn(d, d);
+        acc = (j == 0) ? sq.x : __fmaf_rn(sq.x, one, acc);
+        acc = __fmaf_rn(sq.y, one, acc);
+    }
+    return acc;
+}
+
 struct EncodeConsts {
     float s, ms6, ms4;
     float2 rm;
@@ -184,6 +261,72 @@ __device__ __forceinline__ EncodeConsts encode_consts(float s) {
     c.rm = make_float2(__frcp_rn(c.ms6), __frcp_rn(c.ms4));
     c.fast = s >= kFastMinScale;
     return c;
+}
+
+// One 16-element block, two lanes (this lane: x, 8 elements; lane ^ 1: the
+// other 8; both lanes call it together, the whole warp converged), ab = the
+// block max |x|.  Returns this lane's packed codes (element 2j in the low
+// nibble of byte j) and the chosen E4M3 scale byte.
+struct BlockCodes {
+    uint32_t q;
+    uint32_t sb;
+};
+
+__device__ __forceinline__ BlockCodes encode_block(const float2* x, float ab, const float2* tab,
+                                                   const EncodeConsts& c, float one) {
+    // block scales of both targets: RN(ab / RN(6 s)), RN(ab / RN(4 s))
+    float2 rat;
+    if (c.fast && ab >= kFastMinBlockMax) {
+        const float2 AB = make_float2(ab, ab);
+        const float2 q0 = __fmul2_rn(AB, c.rm);
+        const float2 e = __ffma2_rn(q0, make_float2(-c.ms6, -c.ms4), AB);
+        rat = __ffma2_rn(e, c.rm, q0);
+    } else {
+        rat = ratio_slow(ab, c.ms6, c.ms4);
+    }
+    const uint32_t sbp = cvt_e4m3x2(rat.x, rat.y);
+    const uint32_t sb6 = sbp & 0xFFu, sb4 = sbp >> 8;
+    const float2 t6 = tab[sb6], t4 = tab[sb4];
+    uint32_t q6, q4;
+    bool keep4;
+    if (c.fast) {
+        float2 d6[4], d4[4];
+        q6 = quot_codes(x, t6, d6) ^ 0x88888888u;      // codes of x / D
+        q4 = quot_codes(x, t4, d4) ^ 0x88888888u;
+        const float h6 = sse_estimate(x, d6, t6.x), h4 = sse_estimate(x, d4, t4.x);
+        const float E6 = __fadd_rn(h6, __shfl_xor_sync(0xFFFFFFFFu, h6, 1));
+        const float E4 = __fadd_rn(h4, __shfl_xor_sync(0xFFFFFFFFu, h4, 1));
+        const float diff = __fsub_rn(E4, E6);
+        const float tau = __fmaf_rn(0x1p-16f, __fadd_rn(E4, E6), 0x1p-18f * __fmul_rn(ab, ab));
+        const bool same = sb6 == sb4;          // identical candidates: equal errors, keep 6
+        const bool sure = same || (fabsf(diff) > tau && ab >= kApproxMinBlockMax);
+        keep4 = !same && diff < 0.0f;
+        if (__any_sync(0xFFFFFFFFu, !sure)) {
+            // rare: the definition's sums (elements in order, halves added)
+            const float a6 = sse_exact(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                       x[3].y, q6 ^ 0x88888888u, t6.x, one);
+            const float a4 = sse_exact(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                       x[3].y, q4 ^ 0x88888888u, t4.x, one);
+            const float X6 = __fadd_rn(a6, __shfl_xor_sync(0xFFFFFFFFu, a6, 1));
+            const float X4 = __fadd_rn(a4, __shfl_xor_sync(0xFFFFFFFFu, a4, 1));
+            if (!sure) keep4 = X4 < X6;
+        }
+    } else {
+        const Enc8 r6 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                     x[3].y, t6.x);
+        const Enc8 r4 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                     x[3].y, t4.x);
+        q6 = r6.q;
+        q4 = r4.q;
+        const float E6 = __fadd_rn(r6.err, __shfl_xor_sync(0xFFFFFFFFu, r6.err, 1));
+        const float E4 = __fadd_rn(r4.err, __shfl_xor_sync(0xFFFFFFFFu, r4.err, 1));
+        keep4 = E4 < E6;
+    }
+    BlockCodes r;
+    r.q = keep4 ? q4 : q6;
+    if (!((keep4 ? t4.x : t6.x) > 0.0f)) r.q = 0u;      // a zero step stores +0 codes
+    r.sb = keep4 ? sb4 : sb6;
+    return r;
 }
 
 }  // namespace

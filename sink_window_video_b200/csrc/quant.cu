@@ -8,29 +8,37 @@
 // lower squared error kept; K has its per-head, per-channel mean over the
 // chunk's tokens removed first and kept in fp32.
 //
-// One cooperative persistent kernel per chunk, four phases split by grid
-// barriers.  HBM is read once (K and V, 2 bytes per element); the second
-// read of each tensor hits L2 (126 MB holds both), steered by L2 eviction
-// hints:
-//   A. max |V|:  one streaming pass over V, per-CTA partial maxima.
-//   B. the K column statistics of every (64-token segment, 256-column group)
-//      -- fp32 column sums in token order, bf16 column min and max -- read
-//      from HBM, and the encoding of V (its tensor scale is known after A)
-//      from L2: every warp takes its statistics units first and its V units
-//      after, so each SM interleaves K's HBM stream with V's arithmetic.
-//   C. per column: the segment sums added in segment order and divided by
-//      T (the mean); max |K - mean| from the column min/max (x -> RN(x - mean)
-//      is monotone).
-//   D. the encoding of K from L2.
+// One cooperative persistent kernel per chunk (one CTA of 24 warps per SM).
+// HBM is read once (K and V, 2 bytes per element); the encoding re-reads each
+// tensor from L2 (126 MB holds both), steered by L2 eviction hints.  The CTAs
+// never wait at a grid-wide barrier: they publish their progress in counters
+// of the workspace's control block, and a warp waits (bounded in time) only
+// for the one result it needs next:
+//   1. all warps: max |V| over an even slice of V (read from HBM, kept in
+//      L2); each CTA folds its maximum into a global atomic maximum and counts
+//      itself in.
+//   2. warps 0-7 ("statistics warps"): the K column statistics of the CTA's
+//      (64-token segment, 256-column group) units -- fp32 column sums in
+//      token order, bf16 column minima and maxima -- read from HBM; then, once
+//      every CTA's statistics are in, the mean of the CTA's 32-column blocks
+//      (segment sums added in segment order, / T) and max |K - mean| per
+//      column from its minimum and maximum (x -> RN(x - mean) is monotone),
+//      folded into a global atomic maximum.
+//      warps 8-23, and the statistics warps after that: the encoding of V
+//      (its tensor scale is known once every CTA has counted in), so K's HBM
+//      stream overlaps V's arithmetic on every SM.
+//   3. all warps: the encoding of K, once every column block is finalized.
+// The last CTA to finish resets the counters for the next launch.
 // Encoding: two lanes per 16-element block (8 elements each, one 128-bit
-// load); the block max and the two half-errors meet through one shuffle each.
-// Both targets' block scales come from one paired division, their decoded
-// step D and RN(1/D) from a 256-entry table per tensor, and every division
-// x / D is Markstein's correctly rounded quotient (one multiply, two fused
-// multiply-adds) on float pairs.
+// load), see encode_block (nvfp4_encode.cuh): both targets' scales from one
+// paired division, codes of correctly rounded quotients, the candidates
+// compared on error estimates with the definition's exact sums whenever the
+// estimates are close.
 // Every fp32 step that the definition fixes is one IEEE operation (explicit
 // _rn intrinsics, compiled without FMA contraction), so codes, scales, means
 // and tensor scales are bit-identical to the definition.
+#include <cstddef>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "nvfp4_encode.cuh"
@@ -40,9 +48,14 @@ namespace {
 
 constexpr int kQuantThreads = 768;       // one CTA per SM: 24 warps
 constexpr int kQuantWarps = kQuantThreads / 32;
-constexpr int kEncTokens = 8;          // tokens per encoding unit (one warp)
-constexpr int kFinCols = 32;           // columns per finalize block (one per lane)
-constexpr int kFinSegs = 120;          // segments staged per finalize pass (5 per warp)
+constexpr int kStatsWarps = 8;           // warps 0-7 read K's statistics first
+constexpr int kEncTokens = 16;           // tokens per encoding unit (one warp)
+constexpr int kFinCols = 32;             // columns per finalize block (one per lane)
+constexpr int kStatsBatch = 8;           // K rows in flight per lane in the statistics pass
+constexpr int kFinSegs = 120;            // segments staged per finalize pass
+constexpr int kSegsPerStatsWarp = kFinSegs / kStatsWarps;
+static_assert(kFinSegs % kStatsWarps == 0, "finalize staging splits evenly");
+
 struct QuantArgs {
     const uint4* K;
     const uint4* V;
@@ -62,15 +75,24 @@ struct QuantArgs {
     float one;              // 1 as a run-time value (see encode8_fast)
 };
 
+// Shared memory of the chunk quantizer (the sequence-parallel kernels use the
+// table and the staging areas).
 struct QuantShared {
     float red[kQuantWarps];
-    unsigned qhead;                           // this CTA's phase-B work queue
-    float2 tab[256];                          // per E4M3 code: D = RN(code * s), RN(1/D)
-    uint8_t sb[kQuantWarps][kEncTokens * 8];  // staged scale bytes of one unit per warp
+    float2 tab[2][256];                       // per E4M3 code: D = RN(code * s), RN(1/D); [V, K]
+    float s[2];                               // tensor scales [V, K]
+    int ready[2];                             // tables built (1) or given up (-1)
+    int claim[2];                             // table builder election
+    int abort;                                // a wait of this CTA gave up
+    int fin_go;                               // the statistics warps may finalize
+    unsigned q_stats, q_v, q_k;               // this CTA's work queues
+    alignas(16) uint8_t sb[kQuantWarps][kEncTokens * 8];  // staged scale bytes of a unit per warp
     float fsum[kFinSegs][kFinCols];           // finalize staging
     unsigned short fmin[kFinSegs][kFinCols];
     unsigned short fmax[kFinSegs][kFinCols];
 };
+// a staged row of 8 scale bytes is copied out as one 8-byte word
+static_assert(offsetof(QuantShared, sb) % 16 == 0, "scale staging is 16-byte aligned");
 
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
@@ -91,23 +113,95 @@ __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The tensor scale from the per-CTA partial maxima, and the decode table.
-__device__ __forceinline__ float tensor_scale_and_table(const float* part, QuantShared& sh) {
-    float m = 0.0f;
-    for (int i = threadIdx.x; i < gridDim.x; i += blockDim.x) m = fmaxf(m, __ldcg(part + i));
-    const float A = block_max(m, sh.red);
-    const float s = A > 0.0f ? __fdiv_rn(A, kTensorScaleDiv) : 1.0f;
-    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+// The decode table of one tensor: per E4M3 code c, D = RN(decode(c) * s) and
+// RN(1/D) (0 for D = 0), entries [first, 256) in steps of `step`.
+__device__ __forceinline__ void fill_table(float2* tab, float s, int first, int step) {
+    for (int c = first; c < 256; c += step) {
         const float D = __fmul_rn(e4m3_to_f32((uint32_t)c), s);
-        sh.tab[c] = make_float2(D, D > 0.0f ? __frcp_rn(D) : 0.0f);
+        tab[c] = make_float2(D, D > 0.0f ? __frcp_rn(D) : 0.0f);
     }
-    __syncthreads();
-    return s;
 }
 
-// ---------------------------------------------------------------- phase A
+// ---------------------------------------------------------------- bounded waits
 
-__device__ void phase_vmax(const QuantArgs& a, QuantShared& sh, uint64_t keep) {
+// Wait (one thread) until *counter == target; gives up at the time limit, or
+// at once when this CTA already gave up somewhere.
+__device__ bool wait_counter(const unsigned* counter, unsigned target, Control* ctl,
+                             volatile int* abort, unsigned site) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_acquire_gpu(counter) != target) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_timeout(ctl, site, target, 0u);
+            *abort = 1;
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
+}
+
+// The tensor scale and decode table of V (which = 0) or K (1) in this CTA's
+// shared memory.  The first warp to ask builds it, once the global maximum is
+// complete (every CTA counted in, resp. every column block finalized); the
+// others wait for it.  Returns false when a wait gave up.
+__device__ bool ensure_table(const QuantArgs& a, QuantShared& sh, int which) {
+    volatile int* ready = &sh.ready[which];
+    const int lane = threadIdx.x & 31;
+    int state = *ready;
+    if (state == 0) {
+        int mine = 0;
+        if (lane == 0) mine = atomicCAS(&sh.claim[which], 0, 1) == 0;
+        mine = __shfl_sync(0xFFFFFFFFu, mine, 0);
+        if (mine) {
+            int ok = 1;
+            if (lane == 0) {
+                ok = which == 0 ? wait_counter(&a.ctl->q_vdone, gridDim.x, a.ctl, &sh.abort, 101u)
+                                : wait_counter(&a.ctl->q_fdone, (unsigned)(a.HD / kFinCols),
+                                               a.ctl, &sh.abort, 102u);
+            }
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) {
+                if (lane == 0) *ready = -1;
+                return false;
+            }
+            const float A = __uint_as_float(ld_acquire_gpu(which == 0 ? &a.ctl->q_vmax
+                                                                      : &a.ctl->q_kmax));
+            const float s = A > 0.0f ? __fdiv_rn(A, kTensorScaleDiv) : 1.0f;
+            fill_table(sh.tab[which], s, lane, 32);
+            if (lane == 0) {
+                sh.s[which] = s;
+                if (blockIdx.x == 0) a.tensor_scales[which == 0 ? 1 : 0] = s;
+            }
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) *ready = 1;
+            return true;
+        }
+        if (lane == 0) {
+            // twice the builder's limit: a builder that gives up is the wait recorded
+            const unsigned long long t0 = globaltimer_ns();
+            while ((state = *ready) == 0) {
+                if (sh.abort) break;
+                if (globaltimer_ns() - t0 > 2 * kWaitLimitNs) {
+                    record_timeout(a.ctl, 103u + which, 0u, 0u);
+                    sh.abort = 1;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        state = __shfl_sync(0xFFFFFFFFu, *ready, 0);
+    }
+    __threadfence_block();
+    return state == 1;
+}
+
+// ---------------------------------------------------------------- max |V|
+
+// max |V| over this CTA's even slice (all threads of the CTA), one streaming
+// pass; the CTA's maximum goes to vpart[blockIdx.x] and is returned.
+__device__ float phase_vmax(const QuantArgs& a, QuantShared& sh, uint64_t keep) {
     const size_t n16 = (size_t)a.T * a.HD / 8;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -133,9 +227,8 @@ __device__ void phase_vmax(const QuantArgs& a, QuantShared& sh, uint64_t keep) {
     }
     const float v = fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
     const float b = block_max(v, sh.red);
-    if (threadIdx.x == 0) {
-        a.vpart[blockIdx.x] = b;
-    }
+    if (threadIdx.x == 0) a.vpart[blockIdx.x] = b;
+    return b;
 }
 
 // ---------------------------------------------------------------- K column statistics
@@ -172,12 +265,12 @@ __device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) { mn[j] = 0x7F807F80u; mx[j] = 0xFF80FF80u; }
     int t = 0;
-    for (; t + 16 <= nt; t += 16) {
-        uint4 w[16];
+    for (; t + kStatsBatch <= nt; t += kStatsBatch) {
+        uint4 w[kStatsBatch];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) w[k] = ld_hint(src + (size_t)(t + k) * row8, keep);
+        for (int k = 0; k < kStatsBatch; ++k) w[k] = ld_hint(src + (size_t)(t + k) * row8, keep);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) stats_k_token(w[k], sum, mn, mx);
+        for (int k = 0; k < kStatsBatch; ++k) stats_k_token(w[k], sum, mn, mx);
     }
     for (; t < nt; ++t) stats_k_token(ld_hint(src + (size_t)t * row8, keep), sum, mn, mx);
     float4* ps = reinterpret_cast<float4*>(a.psum + (size_t)s * a.HD + col);
@@ -190,137 +283,136 @@ __device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
 
 // ---------------------------------------------------------------- encoding
 
-// One unit: head h, tokens [t0, t0 + 8) of K (mean subtracted) or V (mean
-// -0: x + (-0) = x exactly, signed zeros included).  Lane = (token parity,
-// 8-channel group); iteration it covers tokens t0 + 2 it + {0, 1}, with the
-// next iteration's 16 bytes loaded ahead.
-__device__ void encode_unit(const QuantArgs& a, QuantShared& sh, bool isK, int h, int t0,
-                            float s, bool fast, float ms6, float ms4, float2 rm,
-                            uint64_t release) {
+// One unit: head h, tokens [t0, t0 + kEncTokens) of K (mean subtracted) or V
+// (mean -0: x + (-0) = x exactly, signed zeros included).  Lane = (token
+// parity, 8-channel group); iteration it covers tokens t0 + 2 it + {0, 1},
+// with the loads of the next two iterations in flight.
+template <bool IS_K>
+__device__ void encode_unit(const QuantArgs& a, const float2* tab, const EncodeConsts& c,
+                            uint8_t* sbst, int h, int t0, uint64_t release) {
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
     const int c8 = lane & 15;                 // 8-channel group of this lane
     const int tsub = lane >> 4;
-    const bool odd = (lane & 1) != 0;         // second half of its 16-block
-    const uint4* src = isK ? a.K : a.V;
     float2 nmu[4];
-    if (isK) {
+    if (IS_K) {
         const float4* mp = reinterpret_cast<const float4*>(a.k_mean + h * kHeadDim + c8 * 8);
         const float4 m0 = __ldcg(mp), m1 = __ldcg(mp + 1);
         nmu[0] = make_float2(-m0.x, -m0.y);
         nmu[1] = make_float2(-m0.z, -m0.w);
         nmu[2] = make_float2(-m1.x, -m1.y);
         nmu[3] = make_float2(-m1.z, -m1.w);
-    } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) nmu[j] = make_float2(-0.0f, -0.0f);
     }
-    uint32_t* codes = reinterpret_cast<uint32_t*>(isK ? a.k_codes : a.v_codes);
-    auto load = [&](int it) {
-        const int t = t0 + 2 * it + tsub;
-        return t < a.T ? ld_hint(src + ((size_t)t * a.H + h) * 16 + c8, release)
-                       : make_uint4(0u, 0u, 0u, 0u);
+    const size_t row2 = (size_t)a.H * 32;                       // uint4 per two tokens
+    const uint4* src = (IS_K ? a.K : a.V) + ((size_t)(t0 + tsub) * a.H + h) * 16 + c8;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(IS_K ? a.k_codes : a.v_codes) +
+                    ((size_t)h * a.T + t0 + tsub) * 16 + c8;
+    uint8_t* sbw = sbst + tsub * 8 + (c8 >> 1);
+    constexpr int kIters = kEncTokens / 2;
+    // a whole unit needs no per-token check; a ragged last unit reads and
+    // writes only its tokens (zeros stand in for the rest)
+    const bool full = t0 + kEncTokens <= a.T;
+    const int nt = a.T - t0 - tsub;
+    auto load = [&](int it, const uint4* p) {
+        return (full || 2 * it < nt) ? ld_hint(p, release) : make_uint4(0u, 0u, 0u, 0u);
     };
-    uint4 wn = load(0);
+    uint4 wa = load(0, src);
+    uint4 wb = load(1, src + row2);
+    const uint4* pf = src + 2 * row2;
 #pragma unroll 1
-    for (int it = 0; it < kEncTokens / 2; ++it) {
-        const uint4 w = wn;
-        if (it + 1 < kEncTokens / 2) wn = load(it + 1);
-        const int t = t0 + 2 * it + tsub;
+    for (int it = 0; it < kIters; ++it) {
+        const uint4 w = wa;
+        wa = wb;
+        if (it + 2 < kIters) {
+            wb = load(it + 2, pf);
+            pf += row2;
+        }
         float2 x[4];
         {
             const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) x[j] = bf16x2_add_f32x2(u[j], nmu[j]);   // RN(K - mean), or V
+            for (int j = 0; j < 4; ++j) {
+                // bf16 -> fp32 exactly (signed zeros kept); K: RN(K - mean)
+                x[j] = make_float2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xFFFF0000u));
+                if (IS_K) x[j] = __fadd2_rn(x[j], nmu[j]);
+            }
         }
         const float ah = max_abs8(x);
         const float ab = fmaxf(ah, __shfl_xor_sync(0xFFFFFFFFu, ah, 1));
-        // block scales of both targets: RN(ab / RN(6 s)), RN(ab / RN(4 s))
-        float2 rat;
-        if (fast && ab >= kFastMinBlockMax) {
-            const float2 AB = make_float2(ab, ab);
-            const float2 q0 = __fmul2_rn(AB, rm);
-            const float2 e = __ffma2_rn(q0, make_float2(-ms6, -ms4), AB);
-            rat = __ffma2_rn(e, rm, q0);
-        } else {
-            rat = ratio_slow(ab, ms6, ms4);
-        }
-        const uint32_t sbp = cvt_e4m3x2(rat.x, rat.y);
-        const uint32_t sb6 = sbp & 0xFFu, sb4 = sbp >> 8;
-        const float2 t6 = sh.tab[sb6], t4 = sh.tab[sb4];
-        uint32_t q6, q4;
-        float e6, e4;
-        if (fast) {
-            encode8_fast(x, t6, a.one, q6, e6);
-            encode8_fast(x, t4, a.one, q4, e4);
-        } else {
-            const Enc8 r6 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y,
-                                         x[3].x, x[3].y, t6.x);
-            const Enc8 r4 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y,
-                                         x[3].x, x[3].y, t4.x);
-            q6 = r6.q; e6 = r6.err;
-            q4 = r4.q; e4 = r4.err;
-        }
-        // block error = (elements 0..7) + (elements 8..15)
-        const float E6 = __fadd_rn(e6, __shfl_xor_sync(0xFFFFFFFFu, e6, 1));
-        const float E4 = __fadd_rn(e4, __shfl_xor_sync(0xFFFFFFFFu, e4, 1));
-        const bool keep4 = E4 < E6;
-        uint32_t q = keep4 ? q4 : q6;
-        if (!((keep4 ? t4.x : t6.x) > 0.0f)) q = 0u;      // a zero step stores +0 codes
-        if (t < a.T) codes[((size_t)h * a.T + t) * 16 + c8] = q;
-        if (!odd) sh.sb[warp][(2 * it + tsub) * 8 + (c8 >> 1)] = (uint8_t)(keep4 ? sb4 : sb6);
+        const BlockCodes bc = encode_block(x, ab, tab, c, a.one);
+        if (full || 2 * it < nt) *dst = bc.q;
+        dst += 32;
+        if ((lane & 1) == 0) *sbw = (uint8_t)bc.sb;
+        sbw += 16;
     }
     __syncwarp();
     if (lane < kEncTokens && t0 + lane < a.T) {
-        uint8_t* scales = isK ? a.k_scales : a.v_scales;
+        uint8_t* scales = IS_K ? a.k_scales : a.v_scales;
         *reinterpret_cast<uint2*>(scales + ((size_t)h * a.T + t0 + lane) * 8) =
-            *reinterpret_cast<const uint2*>(&sh.sb[warp][lane * 8]);
+            *reinterpret_cast<const uint2*>(sbst + lane * 8);
     }
     __syncwarp();
 }
 
-// ---------------------------------------------------------------- phase B
+// ---------------------------------------------------------------- finalize
 
-__device__ void phase_kstats_vencode(const QuantArgs& a, QuantShared& sh, uint64_t keep,
-                                     uint64_t release) {
-    if (threadIdx.x == 0) sh.qhead = 0u;
-    const float sV = tensor_scale_and_table(a.vpart, sh);     // (its barriers publish qhead)
-    if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scales[1] = sV;
-    const EncodeConsts c = encode_consts(sV);
-    // CTA b owns an even slice of the statistics units and of the V units;
-    // its warps take them from a shared-memory queue, statistics first
-    // (memory-bound) and V encoding after (arithmetic), so every SM
-    // interleaves K's HBM stream with V's arithmetic and no warp idles.
-    const int G = gridDim.x, b = blockIdx.x;
-    const int n_stats = a.nseg * a.ngroups;
-    const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
-    const int n_v = a.H * tiles;
-    const int s0 = (int)((long long)n_stats * b / G), s1 = (int)((long long)n_stats * (b + 1) / G);
-    const int v0 = (int)((long long)n_v * b / G), v1 = (int)((long long)n_v * (b + 1) / G);
-    const unsigned n_mine = (unsigned)((s1 - s0) + (v1 - v0));
+// The mean and max |K - mean| of a 32-column block from every segment's
+// statistics: the statistics warps (256 threads, named barrier 1) stage the
+// segments in shared memory, warp 0 adds them in segment order.  Returns
+// (in warp 0) the block's max |K - mean|.
+__device__ float finalize_block(const QuantArgs& a, QuantShared& sh, int b) {
     const int lane = threadIdx.x & 31;
-    unsigned i = 0;
-    if (lane == 0) i = atomicAdd(&sh.qhead, 1u);
-    i = __shfl_sync(0xFFFFFFFFu, i, 0);
-    while (i < n_mine) {
-        unsigned next = 0;
-        if (lane == 0) next = atomicAdd(&sh.qhead, 1u);
-        if ((int)i < s1 - s0) {
-            stats_unit(a, s0 + (int)i, keep);
-        } else {
-            const int u = v0 + (int)i - (s1 - s0);
-            const int h = u / tiles;
-            const int tile = u - h * tiles;
-            encode_unit(a, sh, false, h, tile * kEncTokens, c.s, c.fast, c.ms6, c.ms4, c.rm,
-                               release);
+    const int warp = threadIdx.x >> 5;
+    const int col = b * kFinCols + lane;
+    const unsigned short* pmin = reinterpret_cast<const unsigned short*>(a.pmin);
+    const unsigned short* pmax = reinterpret_cast<const unsigned short*>(a.pmax);
+    float S = 0.0f, mn = INFINITY, mx = -INFINITY;
+    for (int s0 = 0; s0 < a.nseg; s0 += kFinSegs) {
+        const int ns = min(kFinSegs, a.nseg - s0);
+        float ps[kSegsPerStatsWarp];
+        unsigned short pn[kSegsPerStatsWarp], px[kSegsPerStatsWarp];
+#pragma unroll
+        for (int j = 0; j < kSegsPerStatsWarp; ++j) {
+            const int k = warp + j * kStatsWarps;
+            if (k < ns) {
+                const size_t i = (size_t)(s0 + k) * a.HD + col;
+                ps[j] = __ldcg(a.psum + i);
+                pn[j] = __ldcg(pmin + i);
+                px[j] = __ldcg(pmax + i);
+            }
         }
-        i = __shfl_sync(0xFFFFFFFFu, next, 0);
+#pragma unroll
+        for (int j = 0; j < kSegsPerStatsWarp; ++j) {
+            const int k = warp + j * kStatsWarps;
+            if (k < ns) {
+                sh.fsum[k][lane] = ps[j];
+                sh.fmin[k][lane] = pn[j];
+                sh.fmax[k][lane] = px[j];
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kStatsWarps * 32));
+        if (warp == 0) {
+            for (int k = 0; k < ns; ++k) {
+                S = __fadd_rn(S, sh.fsum[k][lane]);
+                mn = fminf(mn, __uint_as_float((uint32_t)sh.fmin[k][lane] << 16));
+                mx = fmaxf(mx, __uint_as_float((uint32_t)sh.fmax[k][lane] << 16));
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kStatsWarps * 32));
     }
+    float kp = 0.0f;
+    if (warp == 0) {
+        const float mu = __fdiv_rn(S, (float)a.T);
+        a.k_mean[col] = mu;
+        kp = fmaxf(fabsf(__fsub_rn(mx, mu)), fabsf(__fsub_rn(mn, mu)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) kp = fmaxf(kp, __shfl_xor_sync(0xFFFFFFFFu, kp, o));
+    }
+    return kp;
 }
 
-// ---------------------------------------------------------------- phase C
-
-__device__ void phase_finalize(const QuantArgs& a, QuantShared& sh) {
+// The finalize of the sequence-parallel path: all warps of a CTA per 32-column
+// block, the CTA's max |K - mean| into kpart[blockIdx.x].
+__device__ void phase_finalize_all(const QuantArgs& a, QuantShared& sh) {
     float kp = 0.0f;
     const int nblocks = a.HD / kFinCols;
     const float Tf = (float)a.T;
@@ -328,16 +420,16 @@ __device__ void phase_finalize(const QuantArgs& a, QuantShared& sh) {
     const int warp = threadIdx.x >> 5;
     const unsigned short* pmin = reinterpret_cast<const unsigned short*>(a.pmin);
     const unsigned short* pmax = reinterpret_cast<const unsigned short*>(a.pmax);
+    constexpr int kPer = kFinSegs / kQuantWarps;
     for (int b = blockIdx.x; b < nblocks; b += gridDim.x) {
         const int col = b * kFinCols + lane;
         float S = 0.0f, mn = INFINITY, mx = -INFINITY;
         for (int s0 = 0; s0 < a.nseg; s0 += kFinSegs) {
             const int ns = min(kFinSegs, a.nseg - s0);
-            // all warps stage the pass's segments, every load in flight at once ...
-            float ps[kFinSegs / kQuantWarps];
-            unsigned short pn[kFinSegs / kQuantWarps], px[kFinSegs / kQuantWarps];
+            float ps[kPer];
+            unsigned short pn[kPer], px[kPer];
 #pragma unroll
-            for (int j = 0; j < kFinSegs / kQuantWarps; ++j) {
+            for (int j = 0; j < kPer; ++j) {
                 const int k = warp + j * kQuantWarps;
                 if (k < ns) {
                     const size_t i = (size_t)(s0 + k) * a.HD + col;
@@ -347,7 +439,7 @@ __device__ void phase_finalize(const QuantArgs& a, QuantShared& sh) {
                 }
             }
 #pragma unroll
-            for (int j = 0; j < kFinSegs / kQuantWarps; ++j) {
+            for (int j = 0; j < kPer; ++j) {
                 const int k = warp + j * kQuantWarps;
                 if (k < ns) {
                     sh.fsum[k][lane] = ps[j];
@@ -356,7 +448,6 @@ __device__ void phase_finalize(const QuantArgs& a, QuantShared& sh) {
                 }
             }
             __syncthreads();
-            // ... and warp 0 adds them in segment order
             if (warp == 0) {
                 for (int k = 0; k < ns; ++k) {
                     S = __fadd_rn(S, sh.fsum[k][lane]);
@@ -376,47 +467,111 @@ __device__ void phase_finalize(const QuantArgs& a, QuantShared& sh) {
     if (threadIdx.x == 0) a.kpart[blockIdx.x] = b;
 }
 
-// ---------------------------------------------------------------- phase D
+// ---------------------------------------------------------------- the kernel
 
-__device__ void phase_kencode(const QuantArgs& a, QuantShared& sh, uint64_t release) {
-    const float sK = tensor_scale_and_table(a.kpart, sh);
-    if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scales[0] = sK;
-    const EncodeConsts c = encode_consts(sK);
-    const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
-    const int nw = gridDim.x * kQuantWarps;
-    const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
-    for (int u = wg; u < a.H * tiles; u += nw) {
-        const int h = u / tiles;
-        const int tile = u - h * tiles;
-        encode_unit(a, sh, true, h, tile * kEncTokens, c.s, c.fast, c.ms6, c.ms4, c.rm, release);
-    }
+// CTA 0 records when it starts and when it passes a few milestones (its first
+// thread, or the warp that reaches them): a per-phase profile of the launch.
+__device__ __forceinline__ void stamp(const QuantArgs& a, int i) {
+    if (blockIdx.x == 0) a.ctl->stamp[i] = globaltimer_ns();
 }
 
-// CTA 0 records when it starts, when it finishes its share of each phase and
-// when it leaves each grid barrier (then the last CTA has arrived): a
-// per-phase profile of the launch.
-__device__ __forceinline__ void stamp(const QuantArgs& a, int i) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) a.ctl->stamp[i] = globaltimer_ns();
+// A warp takes the next item of a CTA queue: index i < n, or -1.
+__device__ __forceinline__ int take(unsigned* q, int n, volatile int* abort) {
+    int i = 0;
+    if ((threadIdx.x & 31) == 0) i = *abort ? n : (int)atomicAdd(q, 1u);
+    i = __shfl_sync(0xFFFFFFFFu, i, 0);
+    return i < n ? i : -1;
 }
 
 __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a) {
     __shared__ QuantShared sh;
     const uint64_t keep = policy_keep(), release = policy_release();
-    stamp(a, 0);
-    phase_vmax(a, sh, keep);
-    stamp(a, 1);
-    if (!grid_barrier(a.ctl)) return;
-    stamp(a, 2);
-    phase_kstats_vencode(a, sh, keep, release);
-    stamp(a, 3);
-    if (!grid_barrier(a.ctl)) return;
-    stamp(a, 4);
-    phase_finalize(a, sh);
-    stamp(a, 5);
-    if (!grid_barrier(a.ctl)) return;
-    stamp(a, 6);
-    phase_kencode(a, sh, release);
-    stamp(a, 7);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int G = gridDim.x, b = blockIdx.x;
+    if (threadIdx.x == 0) {
+        sh.ready[0] = sh.ready[1] = 0;
+        sh.claim[0] = sh.claim[1] = 0;
+        sh.abort = 0;
+        sh.q_stats = sh.q_v = sh.q_k = 0u;
+        stamp(a, 0);
+    }
+    // 1. max |V| (its barriers also publish the initialization above)
+    const float vmax = phase_vmax(a, sh, keep);
+    if (threadIdx.x == 0) {
+        atomicMax(&a.ctl->q_vmax, __float_as_uint(vmax));
+        __threadfence();
+        atomicAdd(&a.ctl->q_vdone, 1u);
+        stamp(a, 1);
+    }
+    // even slices of every kind of unit per CTA
+    const int n_stats = a.nseg * a.ngroups;
+    const int s0 = (int)((long long)n_stats * b / G), s1 = (int)((long long)n_stats * (b + 1) / G);
+    const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
+    const int n_units = a.H * tiles;
+    const int u0 = (int)((long long)n_units * b / G), u1 = (int)((long long)n_units * (b + 1) / G);
+    volatile int* abort = &sh.abort;
+    uint8_t* sbst = sh.sb[warp];
+
+    if (warp < kStatsWarps) {
+        // 2a. K statistics from HBM
+        int done = 0;
+        for (int i; (i = take(&sh.q_stats, s1 - s0, abort)) >= 0; ++done) stats_unit(a, s0 + i, keep);
+        __threadfence();
+        if (lane == 0 && done > 0) atomicAdd(&a.ctl->q_sdone, (unsigned)done);
+        // 2b. this CTA's column blocks, once every CTA's statistics are in
+        const int nfin = a.HD / kFinCols;
+        for (int fb = b; fb < nfin; fb += G) {
+            // thread 0 decides for all statistics warps (a later abort by another
+            // warp must not split them across the named barriers below)
+            if (threadIdx.x == 0)
+                sh.fin_go = wait_counter(&a.ctl->q_sdone, (unsigned)n_stats, a.ctl, abort, 106u);
+            asm volatile("bar.sync 1, %0;" ::"n"(kStatsWarps * 32));
+            if (!sh.fin_go) break;
+            const float kp = finalize_block(a, sh, fb);
+            if (warp == 0 && lane == 0) {
+                atomicMax(&a.ctl->q_kmax, __float_as_uint(kp));
+                __threadfence();
+                atomicAdd(&a.ctl->q_fdone, 1u);
+            }
+        }
+        if (warp == 0 && lane == 0) stamp(a, 2);
+    }
+    // 2c. V from L2
+    if (ensure_table(a, sh, 0)) {
+        if (warp == kStatsWarps && lane == 0) stamp(a, 3);
+        const EncodeConsts c = encode_consts(sh.s[0]);
+        for (int i; (i = take(&sh.q_v, u1 - u0, abort)) >= 0;) {
+            const int u = u0 + i;
+            const int h = u / tiles;
+            encode_unit<false>(a, sh.tab[0], c, sbst, h, (u - h * tiles) * kEncTokens, release);
+        }
+    }
+    // 3. K from L2
+    if (ensure_table(a, sh, 1)) {
+        if (lane == 0) stamp(a, 4);
+        const EncodeConsts c = encode_consts(sh.s[1]);
+        for (int i; (i = take(&sh.q_k, u1 - u0, abort)) >= 0;) {
+            const int u = u0 + i;
+            const int h = u / tiles;
+            encode_unit<true>(a, sh.tab[1], c, sbst, h, (u - h * tiles) * kEncTokens, release);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        stamp(a, 5);
+        __threadfence();
+        if (atomicAdd(&a.ctl->q_exit, 1u) == (unsigned)G - 1u) {
+            // the last CTA: every other CTA is done with the counters
+            a.ctl->q_vdone = 0u;
+            a.ctl->q_vmax = 0u;
+            a.ctl->q_sdone = 0u;
+            a.ctl->q_fdone = 0u;
+            a.ctl->q_kmax = 0u;
+            __threadfence();
+            a.ctl->q_exit = 0u;
+        }
+    }
 }
 
 // ---------------------------------------------------------------- sequence-parallel phases
@@ -443,13 +598,13 @@ __global__ void __launch_bounds__(kQuantThreads, 1) sp_stats_kernel(QuantArgs a,
     const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     const int nw = gridDim.x * kQuantWarps;
     for (int u = wg; u < a.nseg * a.ngroups; u += nw) stats_unit(a, u, keep);
-    phase_vmax(a, sh, keep);                 // per-CTA max |V| into vpart[blockIdx.x] ...
-    if (threadIdx.x == 0) atomicMax(vmax_bits, __float_as_uint(a.vpart[blockIdx.x]));
+    const float b = phase_vmax(a, sh, keep);         // per-CTA max |V| ...
+    if (threadIdx.x == 0) atomicMax(vmax_bits, __float_as_uint(b));
 }
 
 __global__ void __launch_bounds__(kQuantThreads, 1) sp_finalize_kernel(QuantArgs a) {
     __shared__ QuantShared sh;
-    phase_finalize(a, sh);                   // k_mean, per-CTA max |K - mean| in kpart
+    phase_finalize_all(a, sh);               // k_mean, per-CTA max |K - mean| in kpart
 }
 
 // max over the per-CTA partial maxima of |K - mean| and the given max |V|:
@@ -484,20 +639,21 @@ __global__ void __launch_bounds__(kQuantThreads, 1) sp_encode_kernel(QuantArgs a
     __shared__ QuantShared sh;
     const bool isK = blockIdx.y == 1;
     const float st = a.tensor_scales[isK ? 0 : 1];
-    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
-        const float D = __fmul_rn(e4m3_to_f32((uint32_t)c), st);
-        sh.tab[c] = make_float2(D, D > 0.0f ? __frcp_rn(D) : 0.0f);
-    }
+    fill_table(sh.tab[0], st, threadIdx.x, blockDim.x);
     __syncthreads();
     const EncodeConsts c = encode_consts(st);
     const uint64_t release = policy_release();
-    const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
+    const int wg = blockIdx.x * kQuantWarps + warp;
     const int nw = gridDim.x * kQuantWarps;
     const int tiles = (a.T + kEncTokens - 1) / kEncTokens;
     for (int u = wg; u < a.H * tiles; u += nw) {
         const int h = u / tiles;
-        const int tile = u - h * tiles;
-        encode_unit(a, sh, isK, h, tile * kEncTokens, c.s, c.fast, c.ms6, c.ms4, c.rm, release);
+        const int t0 = (u - h * tiles) * kEncTokens;
+        if (isK)
+            encode_unit<true>(a, sh.tab[0], c, sh.sb[warp], h, t0, release);
+        else
+            encode_unit<false>(a, sh.tab[0], c, sh.sb[warp], h, t0, release);
     }
 }
 

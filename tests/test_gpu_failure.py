@@ -1,11 +1,10 @@
 """Failure detection on the GPU without a fault: every wait in the kernels is
 bounded in time (200 ms) and reports through the workspace's status word.  A
-planted arrival count in the quantizer's grid-barrier counter means that no
-arrival completes the first barrier; every CTA waits for a generation that never
-comes, and the kernel must give up,
-record ERR_DEVICE_TIMEOUT with the barrier's site, and leave the context
-usable: after nvfp4kv_workspace_init the same workspace quantizes the chunk
-bit-exactly again."""
+planted count in the quantizer's "CTAs counted into max |V|" word means that
+the count never reaches the grid size; every CTA's V-table builder waits for
+it, and the kernel must give up, record ERR_DEVICE_TIMEOUT with that wait's
+site, and leave the context usable: after nvfp4kv_workspace_init the same
+workspace quantizes the chunk bit-exactly again."""
 import numpy as np
 import pytest
 
@@ -23,12 +22,12 @@ def test_quantizer_barrier_timeout_is_reported_and_recoverable(lib, orc):
     Kd, Vd = dev_bf16(K), dev_bf16(V)
     ws = lib.new_workspace(T, H)
     torch.cuda.synchronize()
-    ws.view(torch.int32)[1] = 1 << 30      # bar_count: no arrival can complete the barrier
+    ws.view(torch.int32)[26] = 1 << 30     # q_vdone: the count can never reach the grid size
     out = lib.ChunkBuffer(T, H)
     lib.quantize_chunk(Kd, Vd, out, ws)
     diag = ws.view(torch.int32)[3:7].cpu().numpy()        # site, block, step, phase
     assert lib.workspace_status(ws) == lib.ERR_DEVICE_TIMEOUT
-    assert diag[0] == 100                  # the grid barrier gave up
+    assert diag[0] == 101                  # the wait for every CTA's max |V| gave up
     assert lib.workspace_status(ws) == lib.OK              # reading cleared the status
     lib.workspace_init(ws)
     out = lib.ChunkBuffer(T, H)
