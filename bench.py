@@ -321,6 +321,7 @@ def run_ours(args, rank, world, local):
     matrix = run_matrix_quant(swv, pool, stream) if not args.no_matrix else None
     dequant = run_dequant(swv, cache, stream) if not args.no_matrix else None
     qonly = run_quantize_only(swv, stream) if not args.no_quantize_only else None
+    fp4q = run_fp4q(swv, cache, pool, O, stream) if not args.no_fp4q else None
 
     rollouts = None
     if not args.no_rollout:
@@ -328,7 +329,7 @@ def run_ours(args, rank, world, local):
 
     return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
                 e2e_ms=e2e_ms, rollouts=rollouts, matrix=matrix, dequant=dequant,
-                quantize_only=qonly,
+                quantize_only=qonly, fp4q=fp4q,
                 attn_launches=swv.attention_launches(len(cache.keyset(0)), T, H, T))
 
 
@@ -420,6 +421,65 @@ def run_dequant(swv, cache, stream, launches=40):
             "bytes_per_launch": nbytes, "achieved": gbs, "unit": "GB/s", "peak": hpeak,
             "frac": gbs / hpeak, "bound": "hbm", "gpu_launches_per_call": 1,
             "traffic": ncu_traffic("dequantize"), "peak_source": f"{src} hbm"}
+
+
+# ------------------------------------------------------------------ FP4-operand attention
+
+# Dense tensor-core throughput of FP4 (kind::mxf4nvf4) over bf16 on B200: 9 vs
+# 2.25 PFLOP/s nominal.
+FP4_OVER_BF16 = 4.0
+
+
+def run_fp4q(swv, cache, pool, O, stream, launches=30):
+    """nvfp4kv_attention_fp4q over the layer step's key set (5 x 7040 keys):
+    the queries quantized to NVFP4, Q K^T on the block-scaled FP4 tensor
+    cores, P V in fp16.  Q rotates over the pool's 4 query tensors; CUDA
+    events around each call (query quantizer + attention kernel (+ merge)).
+    Roofline: the call's tensor time at the measured peaks -- Q K^T's FLOPs at
+    the FP4 rate (measured bf16 x 4, the nominal ratio) plus P V's at the bf16
+    rate -- over the measured time."""
+    import torch
+    peaks, src = load_peaks()
+    T, H, d = CFG["T_c"], CFG["H"], CFG["d"]
+    ids = cache.keyset(0)
+    chunks = [cache.chunk(0, n) for n in ids]
+    qb = swv.Fp4QBuffer(T, H)
+    ws = cache.ws
+    for i in range(3):
+        swv.attention_fp4q(chunks, pool[i % len(pool)][2], O, qb, ws)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(launches)]
+    torch.cuda.synchronize()
+    for i, (e0, e1) in enumerate(ev):
+        e0.record(stream)
+        swv.attention_fp4q(chunks, pool[i % len(pool)][2], O, qb, ws)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if swv.workspace_status(ws) != swv.OK:
+        raise RuntimeError("device status not OK after the FP4-operand attention")
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / launches
+    # how far the FP4 queries move the output from the fp16-product path
+    O16 = torch.empty_like(O)
+    Q = pool[0][2]
+    swv.attention_fp4q(chunks, Q, O, qb, ws)
+    cache.attention(0, Q, O16)
+    torch.cuda.synchronize()
+    rel = float(torch.linalg.vector_norm((O.float() - O16.float())) /
+                torch.linalg.vector_norm(O16.float()))
+    flops = attn_flops()
+    tf = flops / (ms / 1e3) / 1e12
+    timed_ms = ms * launches
+    bpeak, bname = tensor_peak(peaks, src, timed_ms)
+    fp4_peak = bpeak * FP4_OVER_BF16
+    t_ideal = (flops / 2) / (fp4_peak * 1e12) + (flops / 2) / (bpeak * 1e12)
+    return {"kernel": "nvfp4kv_attention_fp4q (query quantizer + attention)",
+            "ms_per_launch": ms, "flops_per_launch": flops, "achieved": tf,
+            "unit": "TFLOP/s", "bound": "tensor",
+            "peak": flops / t_ideal / 1e12,
+            "frac": (t_ideal * 1e3) / ms,
+            "peak_source": f"{bname}; Q K^T at x{FP4_OVER_BF16:g} (FP4 nominal ratio)",
+            "gpu_launches_per_call": swv.attention_fp4q_launches(len(ids), T, H, T),
+            "rel_l2_vs_f16_queries": rel}
 
 
 # ------------------------------------------------------------------ weights / activations
@@ -717,6 +777,8 @@ def build_line(args, r, world, peaks, peak_src):
         line["dequantize"] = r["dequant"]
     if r.get("quantize_only") is not None:
         line["quantize_only"] = r["quantize_only"]
+    if r.get("fp4q") is not None:
+        line["attention_fp4q"] = r["fp4q"]
     return line
 
 
@@ -732,6 +794,7 @@ def main():
     ap.add_argument("--no-rollout", action="store_true")
     ap.add_argument("--no-matrix", action="store_true")
     ap.add_argument("--no-quantize-only", action="store_true")
+    ap.add_argument("--no-fp4q", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -339,6 +339,50 @@ nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
  */
 int nvfp4kv_attention_launches(int n_chunks, int T_c, int H, int d, int T_q);
 
+/*
+ * Bytes of the caller's buffer for the NVFP4 queries of
+ * nvfp4kv_attention_fp4q.  With R = T_q * H and up(x) = x rounded up to a
+ * multiple of 256: E2M1 codes [R][d / 2] at offset 0 (two per byte, the even
+ * element in the low nibble), E4M3 block scales [R][d / 16] at up(R d / 2),
+ * the FP32 tensor scale at up(R d / 2) + up(R d / 16); total that + 256.
+ * 0 for invalid sizes or d != 128.
+ */
+size_t nvfp4kv_fp4q_bytes(int T_q, int H, int d);
+
+/*
+ * Attention with an FP4-operand S = Q K^T (DeepRead page, Method >
+ * 推理基础设施: W4A4 on Blackwell, FP4 GEMMs in place of BF16 ones): the
+ * queries are quantized to NVFP4 as the activation matrix [T_q * H][d]
+ * (16-element blocks along d, Four-Over-Six, one FP32 tensor scale s_Q --
+ * nvfp4kv_quantize_matrix with NVFP4KV_BLOCKS_1D, Method > 训练基础设施), and
+ *   S = s_Q s_K sum_blocks (q_Q sb_Q)(q_K sb_K) + Q_hat . mean
+ * runs on the block-scaled FP4 tensor cores straight from the cache's E2M1
+ * codes and E4M3 block scales; softmax and P V are nvfp4kv_attention's.  The
+ * result is softmax attention with Q replaced by its NVFP4 reconstruction
+ * Q_hat.
+ *   Arguments as nvfp4kv_attention, plus
+ *   q_fp4: device, 256-byte aligned, nvfp4kv_fp4q_bytes(T_q, H, d) bytes,
+ *          caller-owned; written with the quantized queries (readable after
+ *          the call, in the layout nvfp4kv_fp4q_bytes states).
+ *   ws:    a workspace of nvfp4kv_workspace_bytes(T_c, H, d) bytes; the
+ *          query quantizer uses it as its own workspace first (it is at least
+ *          nvfp4kv_matrix_workspace_bytes() long).
+ * Enqueues nvfp4kv_attention_fp4q_launches() kernels; allocates nothing.
+ * Errors as nvfp4kv_attention (ERR_ALIGNMENT also for q_fp4); the status of
+ * the device work (a wait that gave up, a V-scale spread beyond 2^116) is
+ * read with nvfp4kv_workspace_status.  Q_hat . mean is taken in fp32 from the
+ * decoded queries; S's block products are summed by the tensor core in fp32.
+ */
+nvfp4kv_status nvfp4kv_attention_fp4q(const nvfp4kv_chunk_view* chunks, int n_chunks,
+                                      int T_c, int H, int d, const void* Q, int T_q,
+                                      void* O, int o_dtype, float softmax_scale,
+                                      void* q_fp4, void* ws, nvfp4kv_stream_t stream);
+
+/* Kernels one nvfp4kv_attention_fp4q call enqueues: the query quantizer, the
+ * attention kernel, and the merge kernel when the last wave is split (2 or
+ * 3); 0 for invalid sizes.  Host-only. */
+int nvfp4kv_attention_fp4q_launches(int n_chunks, int T_c, int H, int d, int T_q);
+
 /* ------------------------------------------------------------------ cache */
 
 /* Cache shape.  Sinks and window count whole chunks (a chunk = F_c frames of

@@ -70,6 +70,10 @@ def load():
         "nvfp4kv_dequantize": (st, [cv, i32, i32, i32, vp, vp, i32, vp]),
         "nvfp4kv_attention": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp]),
         "nvfp4kv_attention_launches": (i32, [i32, i32, i32, i32, i32]),
+        "nvfp4kv_fp4q_bytes": (sz, [i32, i32, i32]),
+        "nvfp4kv_attention_fp4q": (st, [cv, i32, i32, i32, i32, vp, i32, vp, i32, f32, vp, vp,
+                                        vp]),
+        "nvfp4kv_attention_fp4q_launches": (i32, [i32, i32, i32, i32, i32]),
         "nvfp4kv_matrix_workspace_bytes": (sz, []),
         "nvfp4kv_chunk_stats": (st, [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
         "nvfp4kv_chunk_finalize": (st, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
@@ -376,6 +380,61 @@ def attention(chunks, Q, O, ws, softmax_scale=0.0, stream=None):
                                     _dtype_code(O), float(softmax_scale), _ptr(ws),
                                     _stream(stream)),
            "nvfp4kv_attention")
+
+
+def fp4q_bytes(T_q, H, d=HEAD_DIM) -> int:
+    return int(load().nvfp4kv_fp4q_bytes(T_q, H, d))
+
+
+def _up256(x):
+    return (x + 255) // 256 * 256
+
+
+class Fp4QBuffer:
+    """Device buffer for the NVFP4 queries of attention_fp4q, with views of its
+    parts: codes [T_q * H, d/2], scales [T_q * H, d/16] (uint8), tensor_scale
+    [1] (float32)."""
+
+    def __init__(self, T_q, H, d=HEAD_DIM, device="cuda"):
+        import torch
+        n = fp4q_bytes(T_q, H, d)
+        if n == 0:
+            raise ValueError(f"unsupported query shape ({T_q}, {H}, {d})")
+        self.T_q, self.H, self.d = T_q, H, d
+        self.buf = torch.zeros(n, dtype=torch.uint8, device=device)
+        R = T_q * H
+        o_s = _up256(R * d // 2)
+        o_t = o_s + _up256(R * d // 16)
+        self.codes = self.buf[:R * d // 2].view(R, d // 2)
+        self.scales = self.buf[o_s:o_s + R * d // 16].view(R, d // 16)
+        self.tensor_scale = self.buf[o_t:o_t + 4].view(torch.float32)
+
+    def to_host(self):
+        return dict(codes=self.codes.cpu().numpy(), scales=self.scales.cpu().numpy(),
+                    s=float(self.tensor_scale[0].item()))
+
+
+def attention_fp4q(chunks, Q, O, qbuf: Fp4QBuffer, ws, softmax_scale=0.0, stream=None):
+    """attention with the queries quantized to NVFP4 (into qbuf) and Q K^T on
+    the block-scaled FP4 tensor cores."""
+    views = [c.view if hasattr(c, "view") else c for c in chunks]
+    arr = (ChunkView * max(1, len(views)))(*views)
+    first = chunks[0] if chunks else None
+    T_c = first.T_c if hasattr(first, "T_c") else 0
+    T_q, H, d = Q.shape
+    _check_qo(Q, O, H, d)
+    if (qbuf.T_q, qbuf.H, qbuf.d) != (T_q, H, d):
+        raise ValueError(f"query buffer for ({qbuf.T_q}, {qbuf.H}, {qbuf.d}), "
+                         f"queries of shape {tuple(Q.shape)}")
+    _check(load().nvfp4kv_attention_fp4q(arr, len(views), T_c, H, d, _ptr(Q), T_q, _ptr(O),
+                                         _dtype_code(O), float(softmax_scale), _ptr(qbuf.buf),
+                                         _ptr(ws), _stream(stream)),
+           "nvfp4kv_attention_fp4q")
+
+
+def attention_fp4q_launches(n_chunks, T_c, H, T_q, d=HEAD_DIM) -> int:
+    """Kernels one attention_fp4q call enqueues (2, or 3 with a split tail)."""
+    return int(load().nvfp4kv_attention_fp4q_launches(n_chunks, T_c, H, d, T_q))
 
 
 def check_formats(op, inp, out, n=None, stream=None):

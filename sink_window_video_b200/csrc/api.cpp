@@ -316,6 +316,40 @@ nvfp4kv_status nvfp4kv_attention(const nvfp4kv_chunk_view* chunks, int n_chunks,
                             (cudaStream_t)stream);
 }
 
+size_t nvfp4kv_fp4q_bytes(int T_q, int H, int d) {
+    if (!valid_shape(T_q, H, d) || d != kHeadDimSupported) return 0;
+    return fp4q_layout(T_q, H).total;
+}
+
+nvfp4kv_status nvfp4kv_attention_fp4q(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                      int H, int d, const void* Q, int T_q, void* O,
+                                      int o_dtype, float softmax_scale, void* q_fp4, void* ws,
+                                      nvfp4kv_stream_t stream) {
+    if (!chunks || !Q || !O || !q_fp4 || !ws || T_q <= 0 || !valid_shape(T_c, H, d) ||
+        !valid_shape(T_q, H, d) || (o_dtype != NVFP4KV_F32 && o_dtype != NVFP4KV_BF16))
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (n_chunks <= 0) return NVFP4KV_ERR_EMPTY_KEYSET;
+    if (n_chunks > NVFP4KV_MAX_KEY_CHUNKS) return NVFP4KV_ERR_CAPACITY;
+    for (int i = 0; i < n_chunks; ++i)
+        if (!view_ok(chunks[i])) return NVFP4KV_ERR_INVALID_ARG;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned16(Q) || !aligned16(O) || !aligned256(q_fp4) || !aligned256(ws))
+        return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)d);
+    return launch_attention_fp4(chunks, n_chunks, T_c, H, Q, T_q, O, o_dtype, softmax_scale,
+                                q_fp4, ws, (cudaStream_t)stream);
+}
+
+int nvfp4kv_attention_fp4q_launches(int n_chunks, int T_c, int H, int d, int T_q) {
+    if (n_chunks <= 0 || n_chunks > NVFP4KV_MAX_KEY_CHUNKS || !valid_shape(T_c, H, d) ||
+        d != kHeadDimSupported || T_q <= 0)
+        return 0;
+    const AttnPlan p = attention_plan_tiles(attention_fp4_key_tiles(n_chunks, T_c), H, T_q,
+                                            ws_layout(T_c, H).apart_pairs);
+    return 2 + (p.n_tail > 0 ? 1 : 0);
+}
+
 nvfp4kv_status nvfp4kv_check_formats(int op, const void* in, void* out, size_t n,
                                      nvfp4kv_stream_t stream) {
     if (!in || !out || op < 0 || op > 5) return NVFP4KV_ERR_INVALID_ARG;

@@ -696,7 +696,7 @@ int g_sm_count[64];     // multiprocessor count per device ordinal (0 = not yet 
 // chosen so that the split pieces finish in the fewest rounds per piece
 // length (ties: fewer pieces), bounded by kMaxSplit, by the key tiles and by
 // the workspace's room for partial results.
-AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs) {
+AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, size_t tail_capacity_pairs) {
     AttnPlan p;
     p.pairs_per_head = (T_q + 255) / 256;
     p.n_pairs = H * p.pairs_per_head;
@@ -715,7 +715,6 @@ AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capac
     const int G = g_sm_count[dev];
     const int n_full = (p.n_pairs / G) * G;
     const int n_tail = p.n_pairs - n_full;
-    const int ntiles = n_chunks * ((T_c + kKeysW - 1) / kKeysW);
     if (n_tail == 0 || (size_t)n_tail > tail_capacity_pairs) return p;
     int best_s = 1;
     double best = 1.0;                        // rounds x piece length of the unsplit tail
@@ -732,6 +731,19 @@ AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capac
         p.n_split = best_s;
     }
     return p;
+}
+
+AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs) {
+    return attention_plan_tiles(n_chunks * ((T_c + kKeysW - 1) / kKeysW), H, T_q,
+                                tail_capacity_pairs);
+}
+
+nvfp4kv_status launch_attention_merge(const float* part, const AttnPlan& plan, int T_q, int H,
+                                      void* O, int o_f32, cudaStream_t stream) {
+    const int warps = plan.n_tail * 256;
+    attention_merge_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(
+        part, plan.n_full, plan.n_tail, plan.n_split, plan.pairs_per_head, T_q, H, O, o_f32);
+    return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
 nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
@@ -771,13 +783,7 @@ nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunk
     const int grid = plan.n_full + plan.n_tail * plan.n_split;
     attention_ws_kernel<<<grid, kThreadsW, kSmemW, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
-    if (plan.n_tail > 0) {
-        const int warps = plan.n_tail * 256;
-        attention_merge_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(
-            a.part, plan.n_full, plan.n_tail, plan.n_split, plan.pairs_per_head, T_q, H, O,
-            a.o_f32);
-        if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
-    }
+    if (plan.n_tail > 0) return launch_attention_merge(a.part, plan, T_q, H, O, a.o_f32, stream);
     return NVFP4KV_OK;
 }
 

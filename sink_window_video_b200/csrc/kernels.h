@@ -60,6 +60,26 @@ struct AttnPlan {
     int pairs_per_head, n_pairs, n_full, n_tail, n_split;
 };
 AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs);
+// The same split for a kernel of `ntiles` key tiles per query block.
+AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, size_t tail_capacity_pairs);
+// The second kernel of a split plan: merges the partial rows in `part` into O.
+nvfp4kv_status launch_attention_merge(const float* part, const AttnPlan& plan, int T_q, int H,
+                                      void* O, int o_f32, cudaStream_t stream);
+
+// The queries as NVFP4 rows for the FP4-operand attention: codes
+// [T_q * H][64], block scales [T_q * H][8], the FP32 tensor scale.
+struct Fp4qLayout {
+    size_t codes, scales, scale, total;
+};
+inline Fp4qLayout fp4q_layout(int T_q, int H) {
+    const size_t rows = (size_t)T_q * H;
+    Fp4qLayout L;
+    L.codes = 0;
+    L.scales = align256(rows * 64);
+    L.scale = L.scales + align256(rows * 8);
+    L.total = L.scale + 256;
+    return L;
+}
 
 // The argument checks of nvfp4kv_quantize_chunk, in its order (need_ws: the
 // workspace pointer is checked too); the no-allocation entry point runs the
@@ -102,6 +122,15 @@ nvfp4kv_status launch_check_formats(int op, const void* in, void* out, size_t n,
 nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                    int H, const void* Q, int T_q, void* O, int o_dtype,
                                    float softmax_scale, void* ws, cudaStream_t stream);
+
+// Sink-window attention with the queries quantized to NVFP4 (into q_fp4,
+// laid out by fp4q_layout) and Q K^T on the block-scaled FP4 tensor cores
+// (attention_fp4.cu); the matrix quantizer runs on ws first.
+int attention_fp4_key_tiles(int n_chunks, int T_c);
+nvfp4kv_status launch_attention_fp4(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
+                                    int H, const void* Q, int T_q, void* O, int o_dtype,
+                                    float softmax_scale, void* q_fp4, void* ws,
+                                    cudaStream_t stream);
 
 // Sink-window attention: the warp-specialized tcgen05 kernel (and its merge
 // kernel for split query blocks).

@@ -105,6 +105,38 @@ def test_rejects_bad_arguments_without_device_work(L):
     assert L.nvfp4kv_workspace_init(None, 256, None) == swv.ERR_INVALID_ARG
 
 
+def test_fp4q_entry_checks_and_layout(L):
+    """nvfp4kv_attention_fp4q rejects what nvfp4kv_attention rejects, plus a
+    missing or misaligned query buffer; the buffer size follows the stated
+    layout (codes, scales, each rounded up to 256 bytes, then the scale)."""
+    cv = swv.ChunkView(FAKE, FAKE + 4096, FAKE + 8192, FAKE + 12288, FAKE + 16384, FAKE + 20480)
+    arr = (swv.ChunkView * 1)(cv)
+    f = L.nvfp4kv_attention_fp4q
+    ok = (arr, 1, 32, 2, 128, FAKE, 32, FAKE, 1, 0.0, FAKE, FAKE, None)
+
+    def call(**kw):
+        args = list(ok)
+        for i, v in kw.items():
+            args[int(i[1:])] = v
+        return f(*args)
+    assert call(a1=0) == swv.ERR_EMPTY_KEYSET
+    assert call(a1=33) == swv.ERR_CAPACITY
+    assert call(a10=None) == swv.ERR_INVALID_ARG          # no query buffer
+    assert call(a11=None) == swv.ERR_INVALID_ARG          # no workspace
+    assert call(a8=7) == swv.ERR_INVALID_ARG              # output dtype
+    assert call(a6=0) == swv.ERR_INVALID_ARG              # T_q = 0
+    assert call(a4=96) == swv.ERR_UNSUPPORTED
+    assert call(a10=FAKE + 16) == swv.ERR_ALIGNMENT
+    assert call(a5=FAKE + 4) == swv.ERR_ALIGNMENT
+    up = lambda x: (x + 255) // 256 * 256
+    for T_q, H in [(1, 1), (300, 2), (7040, 24)]:
+        R = T_q * H
+        assert swv.fp4q_bytes(T_q, H) == up(R * 64) + up(R * 8) + 256
+    assert swv.fp4q_bytes(0, 2) == 0 and swv.fp4q_bytes(32, 2, 64) == 0
+    assert L.nvfp4kv_attention_fp4q_launches(0, 32, 2, 128, 32) == 0
+    assert L.nvfp4kv_attention_fp4q_launches(1, 32, 2, 96, 32) == 0
+
+
 def _cache(L, layers, S_g, S_s, W, T=32, H=2):
     cfg = swv.KVCacheConfig(layers, H, 128, T, S_g, S_s, W)
     h = ctypes.c_void_p()

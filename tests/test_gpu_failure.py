@@ -81,3 +81,45 @@ def test_attention_wait_timeout_is_reported_and_recoverable(lib, orc):
     torch.cuda.synchronize()
     assert lib.workspace_status(ws) == lib.OK
     assert_attention_close(host_to_f64(O), orc.attention_f64(qs, Q), "after the timeout")
+
+
+def test_fp4q_attention_wait_timeout_is_reported_and_recoverable(lib, orc):
+    """The same for the FP4-operand attention kernel: its first producer thread
+    of CTA 0 withholds the first tile's arrival; the call reports
+    ERR_DEVICE_TIMEOUT at one of the waits behind it, in CTA 0, and the next
+    call on the re-initialized workspace matches the oracle."""
+    import time
+
+    import torch
+    from gpu_util import assert_attention_close, host_to_f64
+    T_c, H, T_q = 256, 2, 300
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i in range(3):
+        K = synth.k_with_offsets_bf16(180 + i, 0, 0, (T_c, H, 128))
+        V = synth.gaussian_bf16(180 + i, 0, 0, synth.T_V, (T_c, H, 128))
+        b = lib.ChunkBuffer(T_c, H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), b, ws)
+        bufs.append(b)
+        qs.append(orc.quantize_chunk(K, V))
+    Q = synth.gaussian_bf16(189, 0, 0, synth.T_Q, (T_q, H, 128))
+    Qd = dev_bf16(Q)
+    qb = lib.Fp4QBuffer(T_q, H)
+    O = torch.empty((T_q, H, 128), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    ws.view(torch.int32)[7] = 1
+    t0 = time.perf_counter()
+    lib.attention_fp4q(bufs, Qd, O, qb, ws)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    diag = ws.view(torch.int32)[3:7].cpu().numpy()
+    assert lib.workspace_status(ws) == lib.ERR_DEVICE_TIMEOUT
+    assert int(diag[0]) in (10, 11, 30, 42), diag
+    assert int(diag[1]) & 0xFFFF == 0
+    assert 0.15 < elapsed < 5.0
+    lib.workspace_init(ws)
+    lib.attention_fp4q(bufs, Qd, O, qb, ws)
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    assert_attention_close(host_to_f64(O), orc.attention_f64_fp4q(qs, Q), "after the timeout")

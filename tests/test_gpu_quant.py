@@ -47,8 +47,10 @@ def test_tiny_config_bit_exact(lib, orc):
         _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"tiny chunk {c}")
 
 
-@pytest.mark.parametrize("index", [0, 1])
+@pytest.mark.parametrize("index", [0, 1, 9, 19, 33, 47, 58, 71, 86, 99])
 def test_quantize_only_full_size_bit_exact(lib, orc, index):
+    """Ten of the quantize-only workload's 100 chunks (seeds 1..100), spread
+    over the range, bit-exact at full size."""
     K, V = synth.quant_chunk(index)
     out, _ = _gpu_quant(lib, K, V)
     _assert_same(out.to_host(), orc.quantize_chunk(K, V), f"quantize-only chunk {index}")
