@@ -165,7 +165,7 @@ int nvfp4kv_attention_launches(int n_chunks, int T_c, int H, int d, int T_q) {
     if (!valid_shape(T_c, H, d) || n_chunks < 1 || n_chunks > NVFP4KV_MAX_KEY_CHUNKS ||
         T_q <= 0)
         return 0;
-    const AttnPlan p = attention_plan(n_chunks, T_c, H, T_q, ws_layout(T_c, H).apart_pairs);
+    const AttnPlan p = attention_plan(n_chunks, T_c, H, T_q, ws_layout(T_c, H).apart_rows);
     return p.n_tail > 0 ? 2 : 1;
 }
 
@@ -345,8 +345,7 @@ int nvfp4kv_attention_fp4q_launches(int n_chunks, int T_c, int H, int d, int T_q
     if (n_chunks <= 0 || n_chunks > NVFP4KV_MAX_KEY_CHUNKS || !valid_shape(T_c, H, d) ||
         d != kHeadDimSupported || T_q <= 0)
         return 0;
-    const AttnPlan p = attention_plan_tiles(attention_fp4_key_tiles(n_chunks, T_c), H, T_q,
-                                            ws_layout(T_c, H).apart_pairs);
+    const AttnPlan p = attention_fp4_plan(n_chunks, T_c, H, T_q, ws_layout(T_c, H).apart_rows);
     return 2 + (p.n_tail > 0 ? 1 : 0);
 }
 

@@ -689,7 +689,10 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
 
 }  // namespace
 
-int attention_fp4_key_tiles(int n_chunks, int T_c) { return n_chunks * ((T_c + kKeysF - 1) / kKeysF); }
+AttnPlan attention_fp4_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_rows) {
+    return attention_plan_tiles(n_chunks * ((T_c + kKeysF - 1) / kKeysF), H, T_q, 256,
+                                tail_capacity_rows);
+}
 
 nvfp4kv_status launch_attention_fp4(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                     int H, const void* Q, int T_q, void* O, int o_dtype,
@@ -712,8 +715,7 @@ nvfp4kv_status launch_attention_fp4(const nvfp4kv_chunk_view* chunks, int n_chun
     nvfp4kv_status st = launch_quantize_matrix(Q, T_q * H, kHeadDim, NVFP4KV_BLOCKS_1D, q_codes,
                                                q_scales, q_scale, ws, stream);
     if (st != NVFP4KV_OK) return st;
-    const AttnPlan plan = attention_plan_tiles(attention_fp4_key_tiles(n_chunks, T_c), H, T_q,
-                                               L.apart_pairs);
+    const AttnPlan plan = attention_fp4_plan(n_chunks, T_c, H, T_q, L.apart_rows);
     FArgs a;
     for (int i = 0; i < n_chunks; ++i) {
         a.chunk[i].k_codes = chunks[i].k_codes;
@@ -734,7 +736,7 @@ nvfp4kv_status launch_attention_fp4(const nvfp4kv_chunk_view* chunks, int n_chun
     a.o_f32 = o_dtype == NVFP4KV_F32 ? 1 : 0;
     a.scale_log2 = softmax_scale * kLog2eF;
     a.ctl = static_cast<Control*>(ws);
-    a.pairs_per_head = plan.pairs_per_head;
+    a.pairs_per_head = plan.blocks_per_head;
     a.n_full = plan.n_full;
     a.n_split = plan.n_split;
     a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.apart);

@@ -62,6 +62,7 @@ using namespace tc;
 namespace {
 
 constexpr int kKeysW = 128;                 // keys per tile
+constexpr int kRowsW = 256;                 // query rows per CTA (two tiles)
 constexpr int kStages = 2;                  // de-quantized K/V ring depth
 constexpr int kThreadsW = 384;
 constexpr int kDequantWarps = 3;
@@ -97,7 +98,7 @@ struct WsArgs {
     Control* ctl;
     // work split: CTA b < n_full takes query block b whole; later CTAs take
     // key range (b - n_full) % n_split of query block n_full + (b - n_full) / n_split
-    int pairs_per_head, n_full, n_split;
+    int blocks_per_head, n_full, n_split;
     float* part;            // partial results of split blocks
 };
 
@@ -181,8 +182,8 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
     const int pair = split ? a.n_full + piece / a.n_split : item;
     const int q_split = split ? piece % a.n_split : 0;
     const int n_ranges = split ? a.n_split : 1;
-    const int h = pair / a.pairs_per_head;
-    const int m0 = (pair - h * a.pairs_per_head) * 256;
+    const int h = pair / a.blocks_per_head;
+    const int m0 = (pair - h * a.blocks_per_head) * kRowsW;
     const int H = a.H, T_c = a.T_c;
     const int tiles_per_chunk = (T_c + kKeysW - 1) / kKeysW;
     const int ntiles_all = a.n_chunks * tiles_per_chunk;
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
             const float inv = sVmax / l_run;
             // a split block leaves its unnormalized O, running max and row sum
             // (in units where O / l is the output) for the merge kernel
-            float* prow = split ? a.part + ((size_t)piece * 256 + qi * 128 + r) * kPartialFloats
+            float* prow = split ? a.part + ((size_t)piece * kRowsW + qi * 128 + r) * kPartialFloats
                                 : nullptr;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -644,21 +645,22 @@ __global__ void __launch_bounds__(kThreadsW, 1) attention_ws_kernel(const WsArgs
 
 // Merge of a split query block: per row, M = max m_q, O = sum 2^(m_q - M) O_q /
 // sum 2^(m_q - M) l_q over its key ranges q.  One warp per row, four outputs
-// per lane.
+// per lane.  Partial row rr of tail block tp, key range q, at
+// ((tp * n_split + q) * rows + rr) * kPartialFloats.
 __global__ void __launch_bounds__(256) attention_merge_kernel(const float* part, int n_full,
-                                                              int n_tail, int n_split,
-                                                              int pairs_per_head, int T_q, int H,
+                                                              int n_tail, int n_split, int rows,
+                                                              int blocks_per_head, int T_q, int H,
                                                               void* O, int o_f32) {
     const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (w >= n_tail * 256) return;
-    const int tp = w >> 8, rr = w & 255;
-    const int pair = n_full + tp;
-    const int h = pair / pairs_per_head;
-    const int row = (pair - h * pairs_per_head) * 256 + rr;
+    if (w >= n_tail * rows) return;
+    const int tp = w / rows, rr = w - tp * rows;
+    const int blk = n_full + tp;
+    const int h = blk / blocks_per_head;
+    const int row = (blk - h * blocks_per_head) * rows + rr;
     if (row >= T_q) return;
-    const float* base = part + ((size_t)tp * n_split * 256 + rr) * kPartialFloats;
-    const size_t stride = (size_t)256 * kPartialFloats;
+    const float* base = part + ((size_t)tp * n_split * rows + rr) * kPartialFloats;
+    const size_t stride = (size_t)rows * kPartialFloats;
     float M = -INFINITY;
     for (int q = 0; q < n_split; ++q) M = fmaxf(M, base[q * stride + 128]);
     float L = 0.0f;
@@ -690,17 +692,19 @@ int g_sm_count[64];     // multiprocessor count per device ordinal (0 = not yet 
 
 }  // namespace
 
-// The grid: 256-row query blocks (both tiles of a CTA belong to one head),
-// whole blocks in full waves of one CTA per SM; the blocks left over for a
-// last, partial wave are each split into n_split key ranges, with n_split
-// chosen so that the split pieces finish in the fewest rounds per piece
-// length (ties: fewer pieces), bounded by kMaxSplit, by the key tiles and by
-// the workspace's room for partial results.
-AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, size_t tail_capacity_pairs) {
+// The grid: query blocks of block_rows rows of one head, whole blocks in full
+// waves of one CTA per SM; the blocks left over for a last, partial wave are
+// each split into n_split key ranges, with n_split chosen so that the split
+// pieces finish in the fewest rounds per piece length (ties: fewer pieces),
+// bounded by kMaxSplit, by the key tiles and by the workspace's room for
+// partial results.
+AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, int block_rows,
+                              size_t tail_capacity_rows) {
     AttnPlan p;
-    p.pairs_per_head = (T_q + 255) / 256;
-    p.n_pairs = H * p.pairs_per_head;
-    p.n_full = p.n_pairs;
+    p.block_rows = block_rows;
+    p.blocks_per_head = (T_q + block_rows - 1) / block_rows;
+    p.n_blocks = H * p.blocks_per_head;
+    p.n_full = p.n_blocks;
     p.n_tail = 0;
     p.n_split = 1;
     int dev = 0;
@@ -713,9 +717,9 @@ AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, size_t tail_capacity_p
         g_sm_count[dev] = sms;
     }
     const int G = g_sm_count[dev];
-    const int n_full = (p.n_pairs / G) * G;
-    const int n_tail = p.n_pairs - n_full;
-    if (n_tail == 0 || (size_t)n_tail > tail_capacity_pairs) return p;
+    const int n_full = (p.n_blocks / G) * G;
+    const int n_tail = p.n_blocks - n_full;
+    if (n_tail == 0 || (size_t)n_tail * block_rows > tail_capacity_rows) return p;
     int best_s = 1;
     double best = 1.0;                        // rounds x piece length of the unsplit tail
     for (int sp = 2; sp <= kMaxSplit && sp <= ntiles; ++sp) {
@@ -733,16 +737,17 @@ AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, size_t tail_capacity_p
     return p;
 }
 
-AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs) {
-    return attention_plan_tiles(n_chunks * ((T_c + kKeysW - 1) / kKeysW), H, T_q,
-                                tail_capacity_pairs);
+AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_rows) {
+    return attention_plan_tiles(n_chunks * ((T_c + kKeysW - 1) / kKeysW), H, T_q, kRowsW,
+                                tail_capacity_rows);
 }
 
 nvfp4kv_status launch_attention_merge(const float* part, const AttnPlan& plan, int T_q, int H,
                                       void* O, int o_f32, cudaStream_t stream) {
-    const int warps = plan.n_tail * 256;
+    const int warps = plan.n_tail * plan.block_rows;
     attention_merge_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(
-        part, plan.n_full, plan.n_tail, plan.n_split, plan.pairs_per_head, T_q, H, O, o_f32);
+        part, plan.n_full, plan.n_tail, plan.n_split, plan.block_rows, plan.blocks_per_head,
+        T_q, H, O, o_f32);
     return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
@@ -757,7 +762,7 @@ nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunk
         configured = true;
     }
     const WsLayout L = ws_layout(T_c, H);
-    const AttnPlan plan = attention_plan(n_chunks, T_c, H, T_q, L.apart_pairs);
+    const AttnPlan plan = attention_plan(n_chunks, T_c, H, T_q, L.apart_rows);
     WsArgs a;
     for (int i = 0; i < n_chunks; ++i) {
         a.chunk[i].k_codes = chunks[i].k_codes;
@@ -776,7 +781,7 @@ nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunk
     a.o_f32 = o_dtype == NVFP4KV_F32 ? 1 : 0;
     a.scale_log2 = softmax_scale * kLog2eW;
     a.ctl = static_cast<Control*>(ws);
-    a.pairs_per_head = plan.pairs_per_head;
+    a.blocks_per_head = plan.blocks_per_head;
     a.n_full = plan.n_full;
     a.n_split = plan.n_split;
     a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.apart);

@@ -14,11 +14,11 @@ constexpr int kHeadDimSupported = 128;   // head dimension d the kernels support
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Attention work split (see launch_attention_ws): the 256-row query blocks
-// that do not fill a whole wave of CTAs are split into up to kMaxSplit key
-// ranges, whose partial results (per row: 128 fp32 outputs, the running max
-// and the row sum) go to the workspace and are merged by a second kernel.
-constexpr int kMaxTailPairs = 160;   // more than one wave never remains
+// Attention work split (see attention_plan_tiles): the query blocks that do
+// not fill a whole wave of CTAs are split into up to kMaxSplit key ranges,
+// whose partial results (per row: 128 fp32 outputs, the running max and the
+// row sum) go to the workspace and are merged by a second kernel.
+constexpr int kMaxTailPairs = 160;   // 256-row units: more than one wave never remains
 constexpr int kMaxSplit = 8;
 constexpr int kPartialFloats = 132;  // per row: O[128], m, l, 2 pad (16-byte rows)
 
@@ -29,10 +29,11 @@ constexpr int kPartialFloats = 132;  // per row: O[128], m, l, 2 pad (16-byte ro
 //   kpart     float    [kMaxGrid]   per-CTA max |K - mean|
 //   vpart     float    [kMaxGrid]   per-CTA max |V|
 //   (the quantizer uses the workspace up to here: quant_total)
-//   apart     float    [tail pairs * kMaxSplit][256][132]  attention partials,
-//             sized for up to T query rows
+//   apart     float    [tail rows * kMaxSplit][132]  attention partials, room
+//             for apart_rows tail rows (a multiple of 256, at least T rounded
+//             up to 256 per head, at most 160 x 256)
 struct WsLayout {
-    size_t psum, pmin, pmax, kpart, vpart, quant_total, apart, apart_pairs, total;
+    size_t psum, pmin, pmax, kpart, vpart, quant_total, apart, apart_rows, total;
 };
 
 inline WsLayout ws_layout(int T, int H) {
@@ -47,21 +48,24 @@ inline WsLayout ws_layout(int T, int H) {
     L.vpart = off; off += align256(kMaxGrid * 4);
     L.quant_total = off;
     const size_t pairs = (size_t)H * (((size_t)T + 255) / 256);
-    L.apart_pairs = pairs < (size_t)kMaxTailPairs ? pairs : (size_t)kMaxTailPairs;
-    L.apart = off; off += align256(L.apart_pairs * kMaxSplit * 256 * kPartialFloats * 4);
+    L.apart_rows = 256 * (pairs < (size_t)kMaxTailPairs ? pairs : (size_t)kMaxTailPairs);
+    L.apart = off; off += align256(L.apart_rows * kMaxSplit * kPartialFloats * 4);
     L.total = off;
     return L;
 }
 
-// How one attention call is laid out on the GPU: n_full whole 256-row query
-// blocks, then n_tail blocks each split into n_split key ranges (n_split = 1:
-// no split, no second kernel).
+// How one attention call is laid out on the GPU: query blocks of block_rows
+// rows of one head, n_full of them whole, then n_tail blocks each split into
+// n_split key ranges (n_split = 1: no split, no second kernel).  Block b
+// covers head b / blocks_per_head, rows (b % blocks_per_head) * block_rows...
 struct AttnPlan {
-    int pairs_per_head, n_pairs, n_full, n_tail, n_split;
+    int block_rows, blocks_per_head, n_blocks, n_full, n_tail, n_split;
 };
-AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_pairs);
-// The same split for a kernel of `ntiles` key tiles per query block.
-AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, size_t tail_capacity_pairs);
+// The exact attention kernel's plan (attention_ws.cu).
+AttnPlan attention_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_rows);
+// The plan for a kernel of `ntiles` key tiles per query block of block_rows rows.
+AttnPlan attention_plan_tiles(int ntiles, int H, int T_q, int block_rows,
+                              size_t tail_capacity_rows);
 // The second kernel of a split plan: merges the partial rows in `part` into O.
 nvfp4kv_status launch_attention_merge(const float* part, const AttnPlan& plan, int T_q, int H,
                                       void* O, int o_f32, cudaStream_t stream);
@@ -126,7 +130,7 @@ nvfp4kv_status launch_attention_ws(const nvfp4kv_chunk_view* chunks, int n_chunk
 // Sink-window attention with the queries quantized to NVFP4 (into q_fp4,
 // laid out by fp4q_layout) and Q K^T on the block-scaled FP4 tensor cores
 // (attention_fp4.cu); the matrix quantizer runs on ws first.
-int attention_fp4_key_tiles(int n_chunks, int T_c);
+AttnPlan attention_fp4_plan(int n_chunks, int T_c, int H, int T_q, size_t tail_capacity_rows);
 nvfp4kv_status launch_attention_fp4(const nvfp4kv_chunk_view* chunks, int n_chunks, int T_c,
                                     int H, const void* Q, int T_q, void* O, int o_dtype,
                                     float softmax_scale, void* q_fp4, void* ws,

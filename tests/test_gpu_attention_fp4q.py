@@ -109,8 +109,9 @@ def test_ragged_shapes(lib, orc, T_c, T_q, H):
 
 
 def test_split_last_wave(lib, orc):
-    """149 query blocks: one full wave of whole blocks and one block split over
-    key ranges (three kernels: query quantizer, attention, merge)."""
+    """Query rows for a few whole waves of query blocks plus a last wave of a
+    few blocks, which are split over key ranges (three kernels: query
+    quantizer, attention, merge)."""
     T_c, H, T_q = 200, 1, 149 * 256 - 100
     assert lib.attention_fp4q_launches(2, T_c, H, T_q) == 3
     ws = lib.new_workspace(T_c, H)
