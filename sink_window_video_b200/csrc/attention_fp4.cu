@@ -13,9 +13,9 @@
 // the block products summed by the tensor core in fp32.  The output is
 // attention with the queries replaced by their NVFP4 reconstruction.
 //
-// One CTA per SM: a head and 256 query rows (two 128-row tiles in ping-pong),
-// keys in 96-key tiles (the scale-factor layout wants N in multiples of 32,
-// and 2 x 96 S columns leave tensor memory for the scale factors):
+// One CTA per SM: a head and 256 query rows (two 128-row tiles), keys in
+// 96-key tiles (the scale-factor layout wants N in multiples of 32, and
+// 2 x 96 S columns leave tensor memory for the scale factors):
 //   warps 0-7   softmax (thread = row = tensor-memory lane), tile qi = warp / 4;
 //               at the start they stage their tile's FP4 Q and Q scales
 //   warp 8      the MMA issue (lane 0) and lane quarter 0 of the K scales
@@ -23,14 +23,21 @@
 //               the FP4 operand layout and de-quantizes value row j to fp16;
 //               each warp writes its lane quarter of the K scales
 // Tensor memory (512 columns): S0 0..95 | Q scales 96..111 | S1 128..223 |
-// K scales 224..247 (three ring stages) | O0 256..383 | O1 384..511; P (fp16)
-// over the first 48 columns of its S.  A block-scaled operand's scale factors
-// for 128 (or 96) rows and one K = 64 step take 4 columns: row r in column
-// r / 32 at lane r % 32 of every lane quarter, byte = 16-element block.
+// K scales 224..247 (three ring stages) | O0 256..383 | O1 384..511.  A
+// block-scaled operand's scale factors for 128 (or 96) rows and one K = 64
+// step take 4 columns: row r in column r / 32 at lane r % 32 of every lane
+// quarter, byte = 16-element block.
 // Shared memory: Q tiles (FP4, 2 x 8 KB), a three-stage ring of K code tiles
-// (FP4, 6 KB) and V tiles (fp16, 24 KB, 128-byte swizzle, MN-major).
-// The FP4 operands use the no-swizzle K-major layout: 16-byte chunk c of row
-// r at (r / 8) 512 + c 128 + (r % 8) 16.
+// (FP4, 6 KB) and V tiles (fp16, 24 KB, 128-byte swizzle, MN-major), and one
+// P tile per query tile (fp16, 24 KB).  The FP4 operands and P use the
+// no-swizzle K-major layout: 16-byte chunk c of row r at (r / 8) SBO + c 128 +
+// (r % 8) 16 (SBO 512 for 64-byte rows, 1536 for P's 192-byte rows).
+// Because P lives in shared memory, S is free as soon as the softmax has read
+// it: per key tile t the MMA warp issues QK_i(t+1) once tile i has read S_i(t)
+// (s_free), then PV_i(t) once P_i(t) is written (p_full).  The next tile's
+// logits are therefore ready while this tile's exponentials are computed; the
+// softmax waits for PV_i(t-1) (pv_done) only before it rescales O_i or
+// overwrites P_i.
 // Waits, abort path and work split are attention_ws.cu's.
 #include "common.cuh"
 #include "kernels.h"
@@ -57,7 +64,10 @@ constexpr int kVTileB = 2 * kVHalfB;         // fp16 V tile (96 rows x 256 B)
 constexpr int kOffK = 2 * kQTileB;
 constexpr int kOffV = 34 * 1024;             // 1024-byte aligned (128-byte swizzle atoms)
 static_assert(kOffK + kStagesF * kKTileB <= kOffV, "K ring fits below the V ring");
-constexpr size_t kSmemF = kOffV + (size_t)kStagesF * kVTileB + 1024;
+constexpr int kPTileB = 128 * kKeysF * 2;    // fp16 P of one query tile (128 rows x 96 keys)
+constexpr int kOffP = kOffV + kStagesF * kVTileB;          // 106 KB
+static_assert(kOffP % 1024 == 0, "P tiles aligned");
+constexpr size_t kSmemF = kOffP + 2 * (size_t)kPTileB + 1024;
 constexpr float kLog2eF = 1.4426950408889634f;
 constexpr float kRescaleLog2F = 8.0f;
 constexpr float kFarLog2F = 48.0f;
@@ -90,7 +100,9 @@ struct FShared {
     uint64_t kv_full[kStagesF];
     uint64_t kv_empty[kStagesF];
     uint64_t s_full[2];
+    uint64_t s_free[2];      // every row of tile qi has read its S
     uint64_t p_full[2];
+    uint64_t pv_done[2];     // one phase per P V of tile qi
     uint64_t q_ready[2];
     uint64_t o_final;
     uint64_t drain;
@@ -210,6 +222,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
     uint8_t* Qt = base;
     uint8_t* Kt = base + kOffK;
     uint8_t* Vt = base + kOffV;
+    uint8_t* Pt = base + kOffP;                  // [2][P tile], no-swizzle K-major core matrices
 
     if (warp == kMmaWarpF) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -225,7 +238,9 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sh.s_full[i]), 1);
+            mbar_init(smem_u32(&sh.s_free[i]), 128);
             mbar_init(smem_u32(&sh.p_full[i]), 128);
+            mbar_init(smem_u32(&sh.pv_done[i]), 1);
             mbar_init(smem_u32(&sh.q_ready[i]), 128);
         }
         mbar_init(smem_u32(&sh.o_final), 1);
@@ -338,129 +353,104 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 tc_fence_after();
                 const int valid = min(kKeysF, T_c - j0);
+                // the whole S row, then S is free for the next tile's Q K^T
+                uint32_t s[kKeysF];
+                tmem_ld32(tS, s);
+                tmem_ld32(tS + 32, s + 32);
+                tmem_ld32(tS + 64, s + 64);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sh.s_free[qi]));
+                if (valid < kKeysF) {
+#pragma unroll
+                    for (int k = 0; k < kKeysF; ++k)
+                        if (k >= valid) s[k] = __float_as_uint(-INFINITY);
+                }
+                float m8[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    m8[c] = fmax3f(__uint_as_float(s[c]), __uint_as_float(s[c + 8]),
+                                   __uint_as_float(s[c + 16]));
+#pragma unroll
+                for (int k = 24; k < kKeysF; k += 24)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        m8[c] = fmax3f(m8[c], __uint_as_float(s[k + c]),
+                                       fmax3f(__uint_as_float(s[k + 8 + c]), __uint_as_float(s[k + 16 + c]),
+                                              m8[c]));
+                float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                                  fmaxf(m8[6], m8[7]));
+                mx = fmaf(mx, alpha, beta);
+                const bool grow = mx > m_run + kRescaleLog2F || (m_run == -INFINITY && mx > -INFINITY);
+                float corr = 1.0f;
+                if (grow) {
+                    const float m_new = fmaxf(mx, m_run);
+                    corr = ex2f(m_run - m_new);
+                    l_run *= corr;
+                    m_run = m_new;
+                }
+                if (lrV < -kFarLog2F) {
+                    // (rare, chunk-uniform) the denominator from the keys' own
+                    // exponentials
+                    const float bl = beta - lrV - m_run;
+                    float al = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < kKeysF; ++k)
+                        if (k < valid) al += ex2f(fmaf(__uint_as_float(s[k]), alpha, bl));
+                    l_run += al;
+                }
+                const float b2 = beta - m_run;
+                const float2 b22 = make_float2(b2, b2);
                 float2 acc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                                  make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-                // two 48-key halves: S columns 48 hh .. + 47; P (fp16) of half
-                // hh to columns 24 hh .. + 23, over S columns already read
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t s[48];
-                    __syncwarp();
-                    if (hh == 0) {
-                        tmem_ld32(tS, s);
-                        tmem_ld16(tS + 32, s + 32);
+                uint32_t p[kKeysF / 2];
+#pragma unroll
+                for (int k = 0; k < kKeysF / 2; ++k) {
+                    float2 z = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])),
+                                          alpha2, b22);
+                    if ((k & 7) >= 6) {
+                        z = ex2_poly2(z);
                     } else {
-                        tmem_ld16(tS + 48, s);
-                        tmem_ld32(tS + 64, s + 16);
+                        z.x = ex2f(z.x);
+                        z.y = ex2f(z.y);
                     }
-                    tmem_wait_ld();
-                    const int vh = valid - 48 * hh;
-                    if (vh < 48) {
-#pragma unroll
-                        for (int k = 0; k < 48; ++k)
-                            if (k >= vh) s[k] = __float_as_uint(-INFINITY);
-                    }
-                    float m8[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        m8[c] = fmax3f(__uint_as_float(s[c]), __uint_as_float(s[c + 8]),
-                                       __uint_as_float(s[c + 16]));
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        m8[c] = fmax3f(m8[c], __uint_as_float(s[c + 24]),
-                                       fmaxf(__uint_as_float(s[c + 32]), __uint_as_float(s[c + 40])));
-                    float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
-                                      fmaxf(m8[6], m8[7]));
-                    mx = fmaf(mx, alpha, beta);
-                    const bool grow = mx > m_run + kRescaleLog2F || (m_run == -INFINITY && mx > -INFINITY);
-                    float corr = 1.0f;
-                    if (grow) {
-                        const float m_new = fmaxf(mx, m_run);
-                        corr = ex2f(m_run - m_new);
-                        l_run *= corr;
-                        m_run = m_new;
-                    }
-                    if (__any_sync(0xFFFFFFFFu, grow)) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            acc[i].x *= corr;
-                            acc[i].y *= corr;
-                        }
-                        if (o_written) {
-#pragma unroll 1
-                            for (int q = 0; q < 4; ++q) {
-                                uint32_t ov[32];
-                                tmem_ld32(tO + 32 * q, ov);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-                                tmem_st32(tO + 32 * q, ov);
-                            }
-                        }
-                        if (hh == 1) {
-                            tmem_wait_st();
-                            const uint32_t c2 = pack_f16x2(corr, corr);
-                            uint32_t pv[16];
-                            tmem_ld16(tS, pv);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) pv[i] = hmul2_u32(pv[i], c2);
-                            tmem_st16(tS, pv);
-                            tmem_ld8(tS + 16, pv);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) pv[i] = hmul2_u32(pv[i], c2);
-                            tmem_st8(tS + 16, pv);
-                        }
-                    }
-                    if (lrV < -kFarLog2F) {
-                        // (rare, chunk-uniform) the denominator from the keys'
-                        // own exponentials, S re-read from tensor memory
-                        const float bl = beta - lrV - m_run;
-                        float al = 0.0f;
-#pragma unroll 1
-                        for (int q = 0; q < 3; ++q) {
-                            uint32_t sv[16];
-                            tmem_ld16(tS + 48 * hh + 16 * q, sv);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 16; ++k)
-                                if (16 * q + k < vh) al += ex2f(fmaf(__uint_as_float(sv[k]), alpha, bl));
-                        }
-                        l_run += al;
-                    }
-                    const float b2 = beta - m_run;
-                    const float2 b22 = make_float2(b2, b2);
-                    uint32_t p[24];
-#pragma unroll
-                    for (int k = 0; k < 24; ++k) {
-                        float2 z = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])),
-                                              alpha2, b22);
-                        if ((k & 7) >= 6) {
-                            z = ex2_poly2(z);
-                        } else {
-                            z.x = ex2f(z.x);
-                            z.y = ex2f(z.y);
-                        }
-                        acc[k & 3] = __fadd2_rn(acc[k & 3], z);
-                        p[k] = pack_f16x2(z.x, z.y);
-                    }
-                    __syncwarp();
-                    if (hh == 0) {
-                        tmem_st16(tS, p);
-                        tmem_st8(tS + 16, p + 16);
-                    } else {
-                        tmem_st8(tS + 24, p);
-                        tmem_st16(tS + 32, p + 8);
-                    }
+                    acc[k & 3] = __fadd2_rn(acc[k & 3], z);
+                    p[k] = pack_f16x2(z.x, z.y);
                 }
-                tmem_wait_st();
                 if (!(lrV < -kFarLog2F)) {
                     const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
                     const float2 a03 = __fadd2_rn(a01, a23);
                     l_run += (a03.x + a03.y) * inv_rV;
                 }
+                // the previous P V is complete before O is rescaled and P is
+                // overwritten
+                if (t > 0) {
+                    got = wait_or_abort_f(smem_u32(&sh.pv_done[qi]), (uint32_t)((t - 1) & 1), abort,
+                                          a.ctl, 13u + qi, t);
+                    if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                if (__any_sync(0xFFFFFFFFu, grow) && o_written) {
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + 32 * q, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+                        tmem_st32(tO + 32 * q, ov);
+                    }
+                    tmem_wait_st();
+                }
+                // P' to this tile's P buffer: 16-byte chunk c (keys 8c .. 8c + 7)
+                // of row r at (r / 8) 1536 + c 128 + (r % 8) 16
+                uint8_t* prow = Pt + qi * kPTileB + (r >> 3) * 1536 + (r & 7) * 16;
+#pragma unroll
+                for (int c = 0; c < kKeysF / 8; ++c)
+                    *reinterpret_cast<uint4*>(prow + c * 128) =
+                        make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+                fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(p_full);
                 o_written = true;
@@ -614,17 +604,25 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
             }
             __syncwarp();
         };
+        // P V of tile qi: A = P (fp16, shared memory, no swizzle: LBO 128 along
+        // the keys, SBO 1536 per 8 rows), B = V
+        const uint64_t pdesc0 = umma_desc_noswizzle(smem_u32(Pt), 128, 1536);
         auto issue_pv = [&](int qi, int st, bool first) {
             if (lane == 0) {
                 const uint64_t vd = vdesc0 + (uint64_t)((st * kVTileB) >> 4);
+                const uint64_t pd = pdesc0 + (uint64_t)((qi * kPTileB) >> 4);
                 const uint32_t dt = tmem + kColO + 128u * qi;
-                const uint32_t at = tmem + col_s(qi);
 #pragma unroll
                 for (int ks = 0; ks < kKeysF / 16; ++ks)
-                    mma_ts(dt, at + (uint32_t)(ks * 8), vd + (uint64_t)((ks * 2048) >> 4), idesc_pv,
-                           (ks > 0 || !first) ? 1u : 0u);
+                    mma_ss(dt, pd + (uint64_t)((ks * 256) >> 4), vd + (uint64_t)((ks * 2048) >> 4),
+                           idesc_pv, (ks > 0 || !first) ? 1u : 0u);
+                mma_commit(smem_u32(&sh.pv_done[qi]));
             }
             __syncwarp();
+        };
+        auto wait_all = [&](uint64_t* bar, uint32_t parity, unsigned site, int step) {
+            return __all_sync(0xFFFFFFFFu, wait_or_abort_f(smem_u32(bar), parity, abort, a.ctl,
+                                                           site, (unsigned)step));
         };
         bool ok = wait_or_abort_f(smem_u32(&sh.q_ready[0]), 0u, abort, a.ctl, 40u, 0) &&
                   wait_or_abort_f(smem_u32(&sh.q_ready[1]), 0u, abort, a.ctl, 41u, 0);
@@ -633,7 +631,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
         SfbRows sf_next = load_sfb(a, h, t_begin, tiles_per_chunk, lane, ntiles > 0);
         if (ok && ntiles > 0) {
             tc_fence_after();
-            ok = __all_sync(0xFFFFFFFFu, wait_or_abort_f(smem_u32(&sh.kv_full[0]), 0u, abort, a.ctl, 42u, 0));
+            ok = wait_all(&sh.kv_full[0], 0u, 42u, 0);
             if (ok) {
                 tc_fence_after();
                 put_sfb(0, sf_next);
@@ -641,31 +639,34 @@ __global__ void __launch_bounds__(kThreadsF, 1) attention_fp4_kernel(const FArgs
                 issue_qk(1, 0);
             }
         }
+        // Per tile t: the next tile's Q K^T as soon as each query tile has read
+        // its S, then this tile's P V as each P is written.
         for (int t = 0; t < ntiles && ok; ++t) {
             const int st = t % kStagesF;
-            sf_next = load_sfb(a, h, t_begin + t + 1, tiles_per_chunk, lane, t + 1 < ntiles);
-            ok = __all_sync(0xFFFFFFFFu, wait_or_abort_f(smem_u32(&sh.p_full[0]), (uint32_t)(t & 1), abort, a.ctl, 43u, t));
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(0, st, t == 0);
             const bool more = t + 1 < ntiles;
             const int st2 = (t + 1) % kStagesF;
+            sf_next = load_sfb(a, h, t_begin + t + 1, tiles_per_chunk, lane, more);
             if (more) {
-                ok = __all_sync(0xFFFFFFFFu,
-                                wait_or_abort_f(smem_u32(&sh.kv_full[st2]), (uint32_t)(((t + 1) / kStagesF) & 1),
-                                                abort, a.ctl, 44u, t + 1));
+                ok = wait_all(&sh.kv_full[st2], (uint32_t)(((t + 1) / kStagesF) & 1), 44u, t + 1);
                 if (!ok) break;
                 tc_fence_after();
                 put_sfb(t + 1, sf_next);
-                issue_qk(0, st2);
             }
-            ok = __all_sync(0xFFFFFFFFu, wait_or_abort_f(smem_u32(&sh.p_full[1]), (uint32_t)(t & 1), abort, a.ctl, 45u, t));
+            for (int qi = 0; qi < 2 && ok; ++qi) {
+                ok = wait_all(&sh.s_free[qi], (uint32_t)(t & 1), 46u + qi, t);
+                if (!ok) break;
+                tc_fence_after();
+                if (more) issue_qk(qi, st2);
+            }
+            for (int qi = 0; qi < 2 && ok; ++qi) {
+                ok = wait_all(&sh.p_full[qi], (uint32_t)(t & 1), 43u + 2 * qi, t);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(qi, st, t == 0);
+            }
             if (!ok) break;
-            tc_fence_after();
-            issue_pv(1, st, t == 0);
             if (lane == 0) mma_commit(smem_u32(&sh.kv_empty[st]));
             __syncwarp();
-            if (more) issue_qk(1, st2);
         }
         if (lane == 0) {
             if (ok) mma_commit(smem_u32(&sh.o_final));
