@@ -52,11 +52,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source it was taken on: a changed source reports null until it is captured again.
 NCU_TRAFFIC = {
     "attention": ("sink_window_video_b200/csrc/attention_ws.cu",
-                  "43b4b027366a454ad09f5f26b6249269c83917684536fd5377be5b4fa8e97927", 224931072),
+                  "9b32bdc98dc3116b0a96d8fe5309c1a00aabf18bc35389e901e98f84d158d67b", 226354688),
     "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
                   "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
-                 "6a8cb7ce1a56316e2dad4dd9c3ecd74d349d1a1ea48f29dcccb9dfda8cd02dec", 97600000),
+                 "a548141e07c2e12c4fa9cc861b0c70db5a90ae459d898e673508f754e2a129b5", 95029760),
     "dequantize": ("sink_window_video_b200/csrc/dequant.cu",
                    "7dd04c898e146642244e3c647f75a4c6d746e2fad0c7c310a2255267bb2fd8f6", 51334400),
 }
