@@ -57,6 +57,8 @@ NCU_TRAFFIC = {
                   "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
                  "a548141e07c2e12c4fa9cc861b0c70db5a90ae459d898e673508f754e2a129b5", 95029760),
+    "attention_fp4": ("sink_window_video_b200/csrc/attention_fp4.cu",
+                      "385b563baf2156d9f340a5b351f880de978d2ecddd7e92a3ddefc57bd36f4a2b", 194231296),
     "dequantize": ("sink_window_video_b200/csrc/dequant.cu",
                    "7dd04c898e146642244e3c647f75a4c6d746e2fad0c7c310a2255267bb2fd8f6", 51334400),
 }
@@ -479,6 +481,7 @@ def run_fp4q(swv, cache, pool, O, stream, launches=30):
             "frac": (t_ideal * 1e3) / ms,
             "peak_source": f"{bname}; Q K^T at x{FP4_OVER_BF16:g} (FP4 nominal ratio)",
             "gpu_launches_per_call": swv.attention_fp4q_launches(len(ids), T, H, T),
+            "traffic": ncu_traffic("attention_fp4"),
             "rel_l2_vs_f16_queries": rel}
 
 
