@@ -107,6 +107,39 @@ def test_vscale_spread_whole_blocks(lib, orc, mass, log2r):
     _run(lib, orc, mass, log2r, T_c=136, H=4, T_q=37 * 256, seed=500 + log2r)
 
 
+@pytest.mark.parametrize("log2r", [20, 64])
+@pytest.mark.parametrize("mass", ["small", "even", "large"])
+def test_vscale_spread_fp4_queries(lib, orc, mass, log2r):
+    """The FP4-query attention keeps the same per-chunk V-scale reference:
+    checked against the oracle with NVFP4-reconstructed queries, every row."""
+    import torch
+    T_c, H, T_q, seed = 200, 2, 300, 900 + log2r
+    ws = lib.new_workspace(T_c, H)
+    bufs, qs = [], []
+    for i, (v_log2, k0) in enumerate(_case(mass, log2r)):
+        K, V = _chunk(seed + i, T_c, H, v_log2, k0)
+        b = lib.ChunkBuffer(T_c, H)
+        lib.quantize_chunk(dev_bf16(K), dev_bf16(V), b, ws)
+        bufs.append(b)
+        qs.append(orc.quantize_chunk(K, V))
+    Qf = synth.bf16_bits_to_f32(synth.gaussian_bf16(seed + 9, 0, 0, synth.T_Q,
+                                                    (T_q, H, 128))).astype(np.float64)
+    Qf[..., 0] = Q0
+    Q = synth.to_bf16_bits(Qf)
+    ref = orc.attention_f64_fp4q(qs, Q)
+    qb = lib.Fp4QBuffer(T_q, H)
+    O = torch.empty((T_q, H, 128), dtype=torch.float32, device="cuda")
+    lib.attention_fp4q(bufs, dev_bf16(Q), O, qb, ws)
+    torch.cuda.synchronize()
+    assert lib.workspace_status(ws) == lib.OK
+    out = host_to_f64(O)
+    what = f"FP4 queries, {mass} mass, s_V ratio 2^{log2r}"
+    norm = float(np.abs(ref).max())
+    assert_attention_close(out / norm, ref / norm, what)
+    rr = _row_rel(out, ref)
+    assert float(rr.max()) <= 1e-2, f"{what}: worst row rel-L2 {rr.max():.3e}"
+
+
 def test_vscale_spread_beyond_range_is_reported(lib, orc):
     """V scales 2^120 apart exceed what the fp32 softmax sums hold: the call is
     reported as ERR_UNSUPPORTED by the status check (not silently wrong), and
