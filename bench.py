@@ -56,7 +56,7 @@ NCU_TRAFFIC = {
     "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
                   "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
-                 "a548141e07c2e12c4fa9cc861b0c70db5a90ae459d898e673508f754e2a129b5", 95029760),
+                 "ffba28cf4e3a2bc13d72d317f9f51162afdaa58cb295fff9792e1e3d0661758e", 98012416),
     "attention_fp4": ("sink_window_video_b200/csrc/attention_fp4.cu",
                       "385b563baf2156d9f340a5b351f880de978d2ecddd7e92a3ddefc57bd36f4a2b", 194231296),
     "dequantize": ("sink_window_video_b200/csrc/dequant.cu",

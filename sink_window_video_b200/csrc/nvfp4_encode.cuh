@@ -173,56 +173,16 @@ __device__ __noinline__ float2 ratio_slow(float ab, float ms6, float ms4) {
 // ---------------------------------------------------------------- Four-Over-Six block encoder
 //
 // The choice between the two candidates needs their squared errors E6, E4 in
-// the definition's fp32 order only when they are close.  Each candidate's
-// error is first estimated with one fused multiply-add per element,
-// e' = RN(x - dq D), squared and summed in pairs; the estimate differs from
-// the definition's sum E by at most 27.3 u S + 4.2 u ab^2 (u = 2^-24, S the
-// exact sum of the real errors, ab the block max; derived from one rounding
-// per product and sum step and |dq D| <= |x| + |e|).  When |E4' - E6'| is
-// above 2^-16 (E4' + E6') + 2^-18 ab^2 -- several times that bound for the
-// two candidates together -- the estimates decide; otherwise both sums are
-// recomputed in the definition's order.  Codes come from the correctly
-// rounded quotients either way, so the result is the definition's, bit for
-// bit.
+// the definition's fp32 order only when they are close: each candidate's
+// error is first estimated cheaply (encode_block16 below), and when the
+// estimates are within a threshold several times their error bound, both sums
+// are recomputed in the definition's order (sse_exact).  Codes come from the
+// correctly rounded quotients either way, so the result is the definition's,
+// bit for bit.
 
 // Below this block max the estimate's error analysis (no underflow) is not
 // relied on: the exact sums decide.
 constexpr float kApproxMinBlockMax = 0x1p-50f;
-
-// Eight elements against one candidate (D, r = RN(1/D)): the packed codes of
-// -x / D (Markstein's quotient, which keeps the sign of zero) and their
-// decoded values dq' = -sign(x) |dq| as fp32 pairs.
-__device__ __forceinline__ uint32_t quot_codes(const float2* x, float2 Dr, float2* dq) {
-    const float2 NR = make_float2(-Dr.y, -Dr.y);
-    const float2 D2 = make_float2(Dr.x, Dr.x);
-    float y[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 n0 = __fmul2_rn(x[j], NR);
-        const float2 e = __ffma2_rn(n0, D2, x[j]);
-        const float2 n1 = __ffma2_rn(e, NR, n0);
-        y[2 * j] = n1.x;
-        y[2 * j + 1] = n1.y;
-    }
-    uint32_t h[4];
-    const uint32_t q = cvt_e2m1x8_dec(y, h);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) dq[j] = f16x2_to_f32x2(h[j]);
-    return q;
-}
-
-// The estimate of one half block's squared error: sum RN(x + dq' D)^2 in pairs.
-__device__ __forceinline__ float sse_estimate(const float2* x, const float2* dq, float D) {
-    const float2 D2 = make_float2(D, D);
-    float2 e = __ffma2_rn(dq[0], D2, x[0]);
-    float2 acc = __fmul2_rn(e, e);
-#pragma unroll
-    for (int j = 1; j < 4; ++j) {
-        e = __ffma2_rn(dq[j], D2, x[j]);
-        acc = __ffma2_rn(e, e, acc);
-    }
-    return __fadd_rn(acc.x, acc.y);
-}
 
 // The definition's sum for one half block (elements in order): codes q of
 // -x / D, step D.  Out of line: it runs only when the estimates are too close.
@@ -263,18 +223,69 @@ __device__ __forceinline__ EncodeConsts encode_consts(float s) {
     return c;
 }
 
-// One 16-element block, two lanes (this lane: x, 8 elements; lane ^ 1: the
-// other 8; both lanes call it together, the whole warp converged), ab = the
-// block max |x|.  Returns this lane's packed codes (element 2j in the low
-// nibble of byte j) and the chosen E4M3 scale byte.
-struct BlockCodes {
-    uint32_t q;
+// ---------------------------------------------------------------- one lane per block
+//
+// The same encoder with a whole 16-element block in one lane (no shuffles,
+// the block-level work done once).  The error estimate is taken in quotient
+// units: with y = RN(-x / D) (Markstein, as above) and dq the decoded code of
+// x / D, d = RN(dq + y) is one mixed-precision add per element, and
+// E' = RN(D^2) * (sum of d^2, fused multiply-adds on pairs).  Its distance from
+// the definition's sum E is at most 48 u S + 4 u ab^2 (u = 2^-24, S the exact
+// sum of the real errors e, ab the block max): d D = -(e + x eps1)(1 + eps2)
+// gives |d^2 D^2 - e^2| <= 2u |e| |x| + 2u e^2 per element, sum |e| |x| <=
+// ab^2 + 4 S, and the pair sums, the final add and the scaling by D^2 add
+// 10 u S; E itself is within 2u ab^2 + 28 u S of S by the same counting.  The
+// threshold below is the two-lane encoder's, 2^-16 (E4' + E6') + 2^-18 ab^2,
+// more than twice the bound for both candidates together.
+
+// Two f16 (one word, element 2j low) widened exactly and added to an fp32
+// pair, one rounding each: RN(h + c).
+__device__ __forceinline__ float2 f16x2_add_f32x2(uint32_t h2, float2 c) {
+    float lo, hi;
+    asm("{.reg .b16 l, h;\n"
+        "mov.b32 {l, h}, %2;\n"
+        "add.rn.f32.f16 %0, l, %3;\n"
+        "add.rn.f32.f16 %1, h, %4;}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h2), "f"(c.x), "f"(c.y));
+    return make_float2(lo, hi);
+}
+
+// Eight elements against one candidate (D, r = RN(1/D)): the packed codes of
+// x / D (byte j = elements 2j, 2j+1) from Markstein's quotients of -x / D,
+// and the squared quotient-domain residuals added into acc.
+__device__ __forceinline__ uint32_t cand8(const float2* x, float2 Dr, float2& acc) {
+    const float2 NR = make_float2(-Dr.y, -Dr.y);
+    const float2 D2 = make_float2(Dr.x, Dr.x);
+    float2 y[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 n0 = __fmul2_rn(x[j], NR);
+        const float2 e = __ffma2_rn(n0, D2, x[j]);
+        y[j] = __ffma2_rn(e, NR, n0);                    // -RN(x / D)
+    }
+    const float yv[8] = {y[0].x, y[0].y, y[1].x, y[1].y, y[2].x, y[2].y, y[3].x, y[3].y};
+    const uint32_t q = cvt_e2m1x8(yv) ^ 0x88888888u;     // codes of x / D
+    uint32_t h[4];
+    cvt_e2m1x8_to_f16x2(q, h);                           // dq
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 d = f16x2_add_f32x2(h[j], y[j]);    // RN(dq - x / D)
+        acc = __ffma2_rn(d, d, acc);
+    }
+    return q;
+}
+
+struct BlockCodes16 {
+    uint2 q;          // codes of elements 0..7, 8..15
     uint32_t sb;
 };
 
-__device__ __forceinline__ BlockCodes encode_block(const float2* x, float ab, const float2* tab,
-                                                   const EncodeConsts& c, float one) {
-    // block scales of both targets: RN(ab / RN(6 s)), RN(ab / RN(4 s))
+// One 16-element block in this lane (x: 8 pairs, ab = max |x|).  The whole
+// warp calls it together (the rare exact path is decided warp-wide).
+__device__ __forceinline__ BlockCodes16 encode_block16(const float2* x, float ab,
+                                                       const float2* tab,
+                                                       const EncodeConsts& c, float one) {
     float2 rat;
     if (c.fast && ab >= kFastMinBlockMax) {
         const float2 AB = make_float2(ab, ab);
@@ -287,44 +298,49 @@ __device__ __forceinline__ BlockCodes encode_block(const float2* x, float ab, co
     const uint32_t sbp = cvt_e4m3x2(rat.x, rat.y);
     const uint32_t sb6 = sbp & 0xFFu, sb4 = sbp >> 8;
     const float2 t6 = tab[sb6], t4 = tab[sb4];
-    uint32_t q6, q4;
+    uint2 q6, q4;
     bool keep4;
     if (c.fast) {
-        float2 d6[4], d4[4];
-        q6 = quot_codes(x, t6, d6) ^ 0x88888888u;      // codes of x / D
-        q4 = quot_codes(x, t4, d4) ^ 0x88888888u;
-        const float h6 = sse_estimate(x, d6, t6.x), h4 = sse_estimate(x, d4, t4.x);
-        const float E6 = __fadd_rn(h6, __shfl_xor_sync(0xFFFFFFFFu, h6, 1));
-        const float E4 = __fadd_rn(h4, __shfl_xor_sync(0xFFFFFFFFu, h4, 1));
+        float2 a6 = make_float2(0.0f, 0.0f), a4 = make_float2(0.0f, 0.0f);
+        q6.x = cand8(x, t6, a6);
+        q6.y = cand8(x + 4, t6, a6);
+        q4.x = cand8(x, t4, a4);
+        q4.y = cand8(x + 4, t4, a4);
+        const float E6 = __fmul_rn(__fmul_rn(t6.x, t6.x), __fadd_rn(a6.x, a6.y));
+        const float E4 = __fmul_rn(__fmul_rn(t4.x, t4.x), __fadd_rn(a4.x, a4.y));
         const float diff = __fsub_rn(E4, E6);
         const float tau = __fmaf_rn(0x1p-16f, __fadd_rn(E4, E6), 0x1p-18f * __fmul_rn(ab, ab));
         const bool same = sb6 == sb4;          // identical candidates: equal errors, keep 6
         const bool sure = same || (fabsf(diff) > tau && ab >= kApproxMinBlockMax);
         keep4 = !same && diff < 0.0f;
         if (__any_sync(0xFFFFFFFFu, !sure)) {
-            // rare: the definition's sums (elements in order, halves added)
-            const float a6 = sse_exact(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
-                                       x[3].y, q6 ^ 0x88888888u, t6.x, one);
-            const float a4 = sse_exact(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
-                                       x[3].y, q4 ^ 0x88888888u, t4.x, one);
-            const float X6 = __fadd_rn(a6, __shfl_xor_sync(0xFFFFFFFFu, a6, 1));
-            const float X4 = __fadd_rn(a4, __shfl_xor_sync(0xFFFFFFFFu, a4, 1));
-            if (!sure) keep4 = X4 < X6;
+            // rare: the definition's sums (elements in order, the halves added)
+            const float h6a = sse_exact(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                        x[3].y, q6.x ^ 0x88888888u, t6.x, one);
+            const float h6b = sse_exact(x[4].x, x[4].y, x[5].x, x[5].y, x[6].x, x[6].y, x[7].x,
+                                        x[7].y, q6.y ^ 0x88888888u, t6.x, one);
+            const float h4a = sse_exact(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                        x[3].y, q4.x ^ 0x88888888u, t4.x, one);
+            const float h4b = sse_exact(x[4].x, x[4].y, x[5].x, x[5].y, x[6].x, x[6].y, x[7].x,
+                                        x[7].y, q4.y ^ 0x88888888u, t4.x, one);
+            if (!sure) keep4 = __fadd_rn(h4a, h4b) < __fadd_rn(h6a, h6b);
         }
     } else {
-        const Enc8 r6 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
-                                     x[3].y, t6.x);
-        const Enc8 r4 = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
-                                     x[3].y, t4.x);
-        q6 = r6.q;
-        q4 = r4.q;
-        const float E6 = __fadd_rn(r6.err, __shfl_xor_sync(0xFFFFFFFFu, r6.err, 1));
-        const float E4 = __fadd_rn(r4.err, __shfl_xor_sync(0xFFFFFFFFu, r4.err, 1));
-        keep4 = E4 < E6;
+        const Enc8 r6a = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                      x[3].y, t6.x);
+        const Enc8 r6b = encode8_slow(x[4].x, x[4].y, x[5].x, x[5].y, x[6].x, x[6].y, x[7].x,
+                                      x[7].y, t6.x);
+        const Enc8 r4a = encode8_slow(x[0].x, x[0].y, x[1].x, x[1].y, x[2].x, x[2].y, x[3].x,
+                                      x[3].y, t4.x);
+        const Enc8 r4b = encode8_slow(x[4].x, x[4].y, x[5].x, x[5].y, x[6].x, x[6].y, x[7].x,
+                                      x[7].y, t4.x);
+        q6 = make_uint2(r6a.q, r6b.q);
+        q4 = make_uint2(r4a.q, r4b.q);
+        keep4 = __fadd_rn(r4a.err, r4b.err) < __fadd_rn(r6a.err, r6b.err);
     }
-    BlockCodes r;
+    BlockCodes16 r;
     r.q = keep4 ? q4 : q6;
-    if (!((keep4 ? t4.x : t6.x) > 0.0f)) r.q = 0u;      // a zero step stores +0 codes
+    if (!((keep4 ? t4.x : t6.x) > 0.0f)) r.q = make_uint2(0u, 0u);   // a zero step stores +0 codes
     r.sb = keep4 ? sb4 : sb6;
     return r;
 }

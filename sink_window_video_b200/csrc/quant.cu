@@ -17,23 +17,23 @@
 //   1. all warps: max |V| over an even slice of V (read from HBM, kept in
 //      L2); each CTA folds its maximum into a global atomic maximum and counts
 //      itself in.
-//   2. warps 0-7 ("statistics warps"): the K column statistics of the CTA's
+//   2. warps 0-9 ("statistics warps"): the K column statistics of the CTA's
 //      (64-token segment, 256-column group) units -- fp32 column sums in
 //      token order, bf16 column minima and maxima -- read from HBM; then, once
 //      every CTA's statistics are in, the mean of the CTA's 32-column blocks
 //      (segment sums added in segment order, / T) and max |K - mean| per
 //      column from its minimum and maximum (x -> RN(x - mean) is monotone),
 //      folded into a global atomic maximum.
-//      warps 8-23, and the statistics warps after that: the encoding of V
+//      warps 10-23, and the statistics warps after that: the encoding of V
 //      (its tensor scale is known once every CTA has counted in), so K's HBM
 //      stream overlaps V's arithmetic on every SM.
 //   3. all warps: the encoding of K, once every column block is finalized.
 // The last CTA to finish resets the counters for the next launch.
-// Encoding: two lanes per 16-element block (8 elements each, one 128-bit
-// load), see encode_block (nvfp4_encode.cuh): both targets' scales from one
-// paired division, codes of correctly rounded quotients, the candidates
-// compared on error estimates with the definition's exact sums whenever the
-// estimates are close.
+// Encoding: one lane per 16-element block (two 128-bit loads), four tokens of
+// a head per warp and step, see encode_block16 (nvfp4_encode.cuh): both
+// targets' scales from one paired division, codes of correctly rounded
+// quotients, the candidates compared on error estimates with the definition's
+// exact sums whenever the estimates are close.
 // Every fp32 step that the definition fixes is one IEEE operation (explicit
 // _rn intrinsics, compiled without FMA contraction), so codes, scales, means
 // and tensor scales are bit-identical to the definition.
@@ -48,7 +48,7 @@ namespace {
 
 constexpr int kQuantThreads = 768;       // one CTA per SM: 24 warps
 constexpr int kQuantWarps = kQuantThreads / 32;
-constexpr int kStatsWarps = 8;           // warps 0-7 read K's statistics first
+constexpr int kStatsWarps = 10;          // warps 0-9 read K's statistics first
 constexpr int kEncTokens = 16;           // tokens per encoding unit (one warp)
 constexpr int kFinCols = 32;             // columns per finalize block (one per lane)
 constexpr int kStatsBatch = 8;           // K rows in flight per lane in the statistics pass
@@ -285,64 +285,69 @@ __device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
 
 // One unit: head h, tokens [t0, t0 + kEncTokens) of K (mean subtracted) or V
 // (mean -0: x + (-0) = x exactly, signed zeros included).  Lane = (token
-// parity, 8-channel group); iteration it covers tokens t0 + 2 it + {0, 1},
-// with the loads of the next two iterations in flight.
+// within a step, 16-channel block), one block per lane (encode_block16);
+// step it covers tokens t0 + 4 it + {0..3}, with the next step's loads in
+// flight.
 template <bool IS_K>
 __device__ void encode_unit(const QuantArgs& a, const float2* tab, const EncodeConsts& c,
                             uint8_t* sbst, int h, int t0, uint64_t release) {
     const int lane = threadIdx.x & 31;
-    const int c8 = lane & 15;                 // 8-channel group of this lane
-    const int tsub = lane >> 4;
-    float2 nmu[4];
-    if (IS_K) {
-        const float4* mp = reinterpret_cast<const float4*>(a.k_mean + h * kHeadDim + c8 * 8);
-        const float4 m0 = __ldcg(mp), m1 = __ldcg(mp + 1);
-        nmu[0] = make_float2(-m0.x, -m0.y);
-        nmu[1] = make_float2(-m0.z, -m0.w);
-        nmu[2] = make_float2(-m1.x, -m1.y);
-        nmu[3] = make_float2(-m1.z, -m1.w);
-    }
-    const size_t row2 = (size_t)a.H * 32;                       // uint4 per two tokens
-    const uint4* src = (IS_K ? a.K : a.V) + ((size_t)(t0 + tsub) * a.H + h) * 16 + c8;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(IS_K ? a.k_codes : a.v_codes) +
-                    ((size_t)h * a.T + t0 + tsub) * 16 + c8;
-    uint8_t* sbw = sbst + tsub * 8 + (c8 >> 1);
-    constexpr int kIters = kEncTokens / 2;
+    const int blk = lane & 7;                 // 16-channel block of this lane
+    const int tsub = lane >> 3;               // token within a step
+    // K: this lane's 16 channel means, re-read from L1 every step (held in
+    // registers they would push the encoder out of them)
+    const float4* mp = reinterpret_cast<const float4*>(a.k_mean + h * kHeadDim + blk * 16);
+    const size_t row4 = (size_t)a.H * 64;                       // uint4 per four tokens
+    const uint4* src = (IS_K ? a.K : a.V) + ((size_t)(t0 + tsub) * a.H + h) * 16 + blk * 2;
+    uint2* dst = reinterpret_cast<uint2*>(IS_K ? a.k_codes : a.v_codes) +
+                 ((size_t)h * a.T + t0 + tsub) * 8 + blk;
+    uint8_t* sbw = sbst + tsub * 8 + blk;
+    constexpr int kIters = kEncTokens / 4;
     // a whole unit needs no per-token check; a ragged last unit reads and
     // writes only its tokens (zeros stand in for the rest)
     const bool full = t0 + kEncTokens <= a.T;
     const int nt = a.T - t0 - tsub;
-    auto load = [&](int it, const uint4* p) {
-        return (full || 2 * it < nt) ? ld_hint(p, release) : make_uint4(0u, 0u, 0u, 0u);
+    auto load = [&](int it, const uint4* p, uint4& w0, uint4& w1) {
+        if (full || 4 * it < nt) {
+            w0 = ld_hint(p, release);
+            w1 = ld_hint(p + 1, release);
+        } else {
+            w0 = w1 = make_uint4(0u, 0u, 0u, 0u);
+        }
     };
-    uint4 wa = load(0, src);
-    uint4 wb = load(1, src + row2);
-    const uint4* pf = src + 2 * row2;
+    uint4 a0, a1;
+    load(0, src, a0, a1);
+    const uint4* pf = src + row4;
 #pragma unroll 1
     for (int it = 0; it < kIters; ++it) {
-        const uint4 w = wa;
-        wa = wb;
-        if (it + 2 < kIters) {
-            wb = load(it + 2, pf);
-            pf += row2;
+        const uint4 w0 = a0, w1 = a1;
+        if (it + 1 < kIters) {
+            load(it + 1, pf, a0, a1);
+            pf += row4;
         }
-        float2 x[4];
+        float2 x[8];
         {
-            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                // bf16 -> fp32 exactly (signed zeros kept); K: RN(K - mean)
+            for (int j = 0; j < 8; ++j)
+                // bf16 -> fp32 exactly (signed zeros kept)
                 x[j] = make_float2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xFFFF0000u));
-                if (IS_K) x[j] = __fadd2_rn(x[j], nmu[j]);
+            if (IS_K) {
+                // RN(K - mean)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 m = __ldg(mp + k);
+                    x[2 * k] = __fadd2_rn(x[2 * k], make_float2(-m.x, -m.y));
+                    x[2 * k + 1] = __fadd2_rn(x[2 * k + 1], make_float2(-m.z, -m.w));
+                }
             }
         }
-        const float ah = max_abs8(x);
-        const float ab = fmaxf(ah, __shfl_xor_sync(0xFFFFFFFFu, ah, 1));
-        const BlockCodes bc = encode_block(x, ab, tab, c, a.one);
-        if (full || 2 * it < nt) *dst = bc.q;
+        const float ab = fmaxf(max_abs8(x), max_abs8(x + 4));
+        const BlockCodes16 bc = encode_block16(x, ab, tab, c, a.one);
+        if (full || 4 * it < nt) *dst = bc.q;
         dst += 32;
-        if ((lane & 1) == 0) *sbw = (uint8_t)bc.sb;
-        sbw += 16;
+        *sbw = (uint8_t)bc.sb;
+        sbw += 32;
     }
     __syncwarp();
     if (lane < kEncTokens && t0 + lane < a.T) {
