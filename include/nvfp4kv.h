@@ -456,6 +456,29 @@ nvfp4kv_status kvcache_chunk_view(const kvcache* cache, int layer, int64_t chunk
 nvfp4kv_status kvcache_advance(kvcache* cache, int layer, nvfp4kv_chunk_view* out);
 
 /*
+ * Checkpoint and resume of a cache (host bookkeeping; no device access).  A
+ * checkpoint is kvcache_get_state's bytes plus a copy of the pool's
+ * kvcache_pool_bytes() bytes, which the caller makes (and restores) with its
+ * own copies; the workspace holds nothing that outlives a call.
+ * kvcache_state_bytes: the size of the serialized state for this cache's
+ * configuration: a 4-byte tag "NVKV", a uint32 format version (1), the seven
+ * int32 fields of kvcache_config, the shot sink's first chunk (int64), the
+ * chunks appended per layer (int64 [layers]) and the chunk id held by every
+ * slot (int64 [layers][S_g + S_s + W, at least 1], -1 for a free slot), in
+ * host byte order.
+ * kvcache_get_state writes it into buf (host, at least kvcache_state_bytes).
+ * kvcache_set_state replaces the bookkeeping of a cache created with the same
+ * configuration, over a pool that holds the saved pool's bytes.  It returns
+ * NVFP4KV_ERR_INVALID_ARG and changes nothing if the buffer is short or not
+ * this format, the configuration differs, or the state is inconsistent (a
+ * negative count or shot-sink chunk, a slot holding a chunk outside
+ * [0, count), a chunk held by two slots of a layer).
+ */
+size_t kvcache_state_bytes(const kvcache* cache);
+nvfp4kv_status kvcache_get_state(const kvcache* cache, void* buf, size_t bytes);
+nvfp4kv_status kvcache_set_state(kvcache* cache, const void* buf, size_t bytes);
+
+/*
  * Sink-window attention of `layer`'s queries Q [T_q][H][d] (bf16, device)
  * over its current key set, written to O [T_q][H][d] (device, o_dtype): the
  * key set of kvcache_keyset() passed to nvfp4kv_attention().

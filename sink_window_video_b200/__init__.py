@@ -90,6 +90,9 @@ def load():
         "kvcache_num_chunks": (st, [vp, i32, ctypes.POINTER(i64)]),
         "kvcache_chunk_view": (st, [vp, i32, i64, cv]),
         "kvcache_advance": (st, [vp, i32, cv]),
+        "kvcache_state_bytes": (sz, [vp]),
+        "kvcache_get_state": (st, [vp, vp, sz]),
+        "kvcache_set_state": (st, [vp, vp, sz]),
         "sink_window_attention": (st, [vp, i32, vp, i32, vp, i32, f32, vp]),
         "kvcache_check_status": (st, [vp, vp]),
         "nvfp4kv_check_formats": (st, [i32, vp, vp, sz, vp]),
@@ -519,6 +522,21 @@ class KVCache:
 
     def check_status(self, stream=None) -> int:
         return int(load().kvcache_check_status(self._h, _stream(stream)))
+
+    def get_state(self) -> bytes:
+        """The cache's bookkeeping (kvcache_get_state); with a copy of
+        self.pool it is a checkpoint."""
+        L = load()
+        n = int(L.kvcache_state_bytes(self._h))
+        buf = ctypes.create_string_buffer(n)
+        _check(L.kvcache_get_state(self._h, buf, n), "kvcache_get_state")
+        return buf.raw
+
+    def set_state(self, state: bytes):
+        """Restore bookkeeping saved by get_state (self.pool must hold the saved
+        pool's bytes)."""
+        buf = ctypes.create_string_buffer(state, len(state))
+        _check(load().kvcache_set_state(self._h, buf, len(state)), "kvcache_set_state")
 
 
 def default_scale(d=HEAD_DIM):

@@ -451,6 +451,70 @@ nvfp4kv_status kvcache_advance(kvcache* cache, int layer, nvfp4kv_chunk_view* ou
     return NVFP4KV_ERR_CAPACITY;    // unreachable: the live set fits the pool
 }
 
+namespace {
+constexpr uint32_t kStateVersion = 1;
+constexpr size_t kStateHeader = 4 + 4 + 7 * 4 + 8;      // tag, version, config, shot sink
+}  // namespace
+
+size_t kvcache_state_bytes(const kvcache* cache) {
+    if (!cache) return 0;
+    return kStateHeader + 8 * (size_t)cache->cfg.layers * (1 + (size_t)cache->slots);
+}
+
+nvfp4kv_status kvcache_get_state(const kvcache* cache, void* buf, size_t bytes) {
+    if (!cache || !buf || bytes < kvcache_state_bytes(cache)) return NVFP4KV_ERR_INVALID_ARG;
+    uint8_t* p = static_cast<uint8_t*>(buf);
+    std::memcpy(p, "NVKV", 4);
+    std::memcpy(p + 4, &kStateVersion, 4);
+    const int32_t cfg[7] = {cache->cfg.layers, cache->cfg.H, cache->cfg.d, cache->cfg.T_c,
+                            cache->cfg.S_g,    cache->cfg.S_s, cache->cfg.W};
+    std::memcpy(p + 8, cfg, sizeof(cfg));
+    std::memcpy(p + 36, &cache->s_begin, 8);
+    std::memcpy(p + kStateHeader, cache->n.data(), 8 * cache->n.size());
+    std::memcpy(p + kStateHeader + 8 * cache->n.size(), cache->slot_chunk.data(),
+                8 * cache->slot_chunk.size());
+    return NVFP4KV_OK;
+}
+
+nvfp4kv_status kvcache_set_state(kvcache* cache, const void* buf, size_t bytes) {
+    if (!cache || !buf || bytes < kvcache_state_bytes(cache)) return NVFP4KV_ERR_INVALID_ARG;
+    const uint8_t* p = static_cast<const uint8_t*>(buf);
+    uint32_t version = 0;
+    std::memcpy(&version, p + 4, 4);
+    if (std::memcmp(p, "NVKV", 4) != 0 || version != kStateVersion) return NVFP4KV_ERR_INVALID_ARG;
+    int32_t cfg[7];
+    std::memcpy(cfg, p + 8, sizeof(cfg));
+    const int32_t want[7] = {cache->cfg.layers, cache->cfg.H, cache->cfg.d, cache->cfg.T_c,
+                             cache->cfg.S_g,    cache->cfg.S_s, cache->cfg.W};
+    if (std::memcmp(cfg, want, sizeof(cfg)) != 0) return NVFP4KV_ERR_INVALID_ARG;
+    kvcache next = *cache;
+    std::memcpy(&next.s_begin, p + 36, 8);
+    std::memcpy(next.n.data(), p + kStateHeader, 8 * next.n.size());
+    std::memcpy(next.slot_chunk.data(), p + kStateHeader + 8 * next.n.size(),
+                8 * next.slot_chunk.size());
+    if (next.s_begin < 0) return NVFP4KV_ERR_INVALID_ARG;
+    for (int layer = 0; layer < next.cfg.layers; ++layer) {
+        // (a slot may still hold a chunk that left the key set at a shot-sink
+        // rebind: the next append frees it)
+        const int64_t n = next.n[layer];
+        if (n < 0) return NVFP4KV_ERR_INVALID_ARG;
+        const int64_t* sc = &next.slot_chunk[(size_t)layer * next.slots];
+        std::vector<int64_t> held;
+        for (int s = 0; s < next.slots; ++s) {
+            if (sc[s] == -1) continue;
+            if (sc[s] < 0 || sc[s] >= n) return NVFP4KV_ERR_INVALID_ARG;
+            held.push_back(sc[s]);
+        }
+        std::sort(held.begin(), held.end());
+        if (std::adjacent_find(held.begin(), held.end()) != held.end())
+            return NVFP4KV_ERR_INVALID_ARG;
+    }
+    cache->s_begin = next.s_begin;
+    cache->n = next.n;
+    cache->slot_chunk = next.slot_chunk;
+    return NVFP4KV_OK;
+}
+
 nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const void* V,
                               nvfp4kv_stream_t stream) {
     if (!cache || !K || !V) return NVFP4KV_ERR_INVALID_ARG;

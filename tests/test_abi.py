@@ -260,3 +260,95 @@ def test_noalloc_refuses_every_bad_argument_as_the_workspace_entry_point(L):
         na_status = L.nvfp4kv_quantize_chunk_noalloc(a["K"], a["V"], a["T"], a["H"], a["d"],
                                                      out, None)
         assert ws_status != swv.OK and na_status == ws_status, (c, ws_status, na_status)
+
+
+def _views(L, h, layers):
+    out = []
+    for layer in range(layers):
+        ids = _keyset(L, h, layer)
+        n = ctypes.c_int64()
+        assert L.kvcache_num_chunks(h, layer, ctypes.byref(n)) == swv.OK
+        vs = []
+        for c in ids:
+            v = swv.ChunkView()
+            assert L.kvcache_chunk_view(h, layer, c, ctypes.byref(v)) == swv.OK
+            vs.append((c, v.k_codes, v.v_codes, v.k_scales, v.v_scales, v.k_mean, v.tensor_scales))
+        out.append((n.value, ids, vs))
+    return out
+
+
+def _state(L, h):
+    n = L.kvcache_state_bytes(h)
+    buf = ctypes.create_string_buffer(n)
+    assert L.kvcache_get_state(h, buf, n) == swv.OK
+    return bytearray(buf.raw)
+
+
+def _set(L, h, state):
+    buf = ctypes.create_string_buffer(bytes(state), len(state))
+    return L.kvcache_set_state(h, buf, len(state))
+
+
+def test_cache_state_round_trip(L):
+    """kvcache_get_state / kvcache_set_state: a second cache over the same pool,
+    given the first one's state at random points of a schedule with shot
+    switches, holds the same chunks in the same slots, and both evolve alike
+    afterwards."""
+    rng = random.Random(11)
+    for trial in range(20):
+        layers = rng.randint(1, 3)
+        S_g, S_s, W = rng.randint(0, 2), rng.randint(0, 2), rng.randint(1, 4)
+        h1, cfg = _cache(L, layers, S_g, S_s, W)
+        h2, _ = _cache(L, layers, S_g, S_s, W)
+        assert L.kvcache_state_bytes(h1) == 44 + 8 * layers * (1 + max(1, S_g + S_s + W))
+        n = [0] * layers
+        for step in range(rng.randint(3, 25)):
+            if rng.random() < 0.2 and step > 0:
+                first = max(n)
+                assert L.kvcache_rebind_shot_sink(h1, first) == swv.OK
+                assert L.kvcache_rebind_shot_sink(h2, first) == swv.OK
+            layer = rng.randrange(layers)
+            v1, v2 = swv.ChunkView(), swv.ChunkView()
+            assert L.kvcache_advance(h1, layer, ctypes.byref(v1)) == swv.OK
+            assert L.kvcache_advance(h2, layer, ctypes.byref(v2)) == swv.OK
+            n[layer] += 1
+            if rng.random() < 0.3:
+                assert _set(L, h2, _state(L, h1)) == swv.OK
+                assert _views(L, h2, layers) == _views(L, h1, layers)
+                assert _state(L, h2) == _state(L, h1)
+        assert _views(L, h2, layers) == _views(L, h1, layers)
+        L.kvcache_destroy(h1)
+        L.kvcache_destroy(h2)
+
+
+def test_cache_state_refusals_change_nothing(L):
+    h, cfg = _cache(L, 2, 1, 1, 3)
+    for layer in (0, 1, 0, 0):
+        v = swv.ChunkView()
+        assert L.kvcache_advance(h, layer, ctypes.byref(v)) == swv.OK
+    good = _state(L, h)
+    other, _ = _cache(L, 2, 1, 1, 4)
+    slots = 5
+    n_off, s_off = 44, 44 + 16                 # counts of 2 layers, then the slot map
+
+    def put64(st, off, v):
+        st[off:off + 8] = int(v).to_bytes(8, "little", signed=True)
+
+    bad = []
+    bad.append(good[:-1])                                       # short
+    b = bytearray(good); b[0:4] = b"NVKX"; bad.append(b)        # not this format
+    b = bytearray(good); b[4] = 2; bad.append(b)                # another version
+    b = bytearray(good); b[8 + 6 * 4] = 9; bad.append(b)        # another window
+    b = bytearray(good); put64(b, n_off, -1); bad.append(b)     # negative count
+    b = bytearray(good); put64(b, 36, -3); bad.append(b)        # negative shot sink
+    b = bytearray(good); put64(b, s_off, 7); bad.append(b)      # a chunk never appended
+    b = bytearray(good)
+    put64(b, s_off, 1); put64(b, s_off + 8, 1); bad.append(b)   # one chunk in two slots
+    before = _views(L, h, 2)
+    for st in bad:
+        assert _set(L, h, st) == swv.ERR_INVALID_ARG
+        assert _state(L, h) == good and _views(L, h, 2) == before
+    assert _set(L, other, good) == swv.ERR_INVALID_ARG          # another configuration
+    assert _set(L, h, good) == swv.OK
+    L.kvcache_destroy(h)
+    L.kvcache_destroy(other)
