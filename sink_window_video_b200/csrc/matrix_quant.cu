@@ -8,8 +8,8 @@
 //
 // One cooperative persistent kernel, two phases split by a grid barrier:
 //   A. max |X|: one streaming pass (L2 evict_last), per-CTA partial maxima;
-//   B. the encoding, X re-read from L2 (evict_first): 1D -- one warp per
-//      256-column row segment, two lanes per block; 2D -- one warp per tile,
+//   B. the encoding, X re-read from L2 (evict_first): 1D -- 32 consecutive
+//      blocks per warp, one lane per block; 2D -- one warp per tile,
 //      lane = (row, half row).
 // The block arithmetic is the KV quantizer's (nvfp4_encode.cuh), bit-identical
 // to the definition.
@@ -126,33 +126,32 @@ __device__ __forceinline__ void load_x(const uint4& w, float2* x) {
     for (int j = 0; j < 4; ++j) x[j] = bf16x2_add_f32x2(u[j], nz);
 }
 
-// 1D: one 256-column segment of one row; lanes 2k, 2k+1 hold block k.
+// 1D: 32 consecutive 16-element blocks of the dense [M][N] matrix per warp and
+// step (block b = elements 16 b .. 16 b + 15, a row's blocks followed by the
+// next row's since N % 16 == 0), one block per lane (encode_block16: the
+// block-level work once, no shuffles): 1 KB contiguous per warp for any N.
 __device__ void encode_rows(const MatArgs& a, const MatShared& sh, const EncodeConsts& c,
                             uint64_t release) {
     const int lane = threadIdx.x & 31;
-    const int wg = blockIdx.x * kMqWarps + (threadIdx.x >> 5);
-    const int nw = gridDim.x * kMqWarps;
-    const int segs = (a.N + 255) / 256;
-    const bool odd = (lane & 1) != 0;
-    for (int u = wg; u < a.M * segs; u += nw) {
-        const int row = u / segs;
-        const int col = (u - row * segs) * 256 + lane * 8;
-        const bool valid = col < a.N;                         // both lanes of a block alike
-        const size_t e0 = (size_t)row * a.N + col;
-        float2 x[4];
-        load_x(valid ? ld_hint(a.X + e0 / 8, release) : make_uint4(0u, 0u, 0u, 0u), x);
-        const float ah = max_abs8(x);
-        const float ab = fmaxf(ah, __shfl_xor_sync(0xFFFFFFFFu, ah, 1));
-        const LaneEnc r = encode_lane(x, ab, sh, c, a.one);
-        // block error = (elements 0..7) + (elements 8..15)
-        const float E6 = __fadd_rn(r.e6, __shfl_xor_sync(0xFFFFFFFFu, r.e6, 1));
-        const float E4 = __fadd_rn(r.e4, __shfl_xor_sync(0xFFFFFFFFu, r.e4, 1));
-        const bool keep4 = E4 < E6;
-        uint32_t q = keep4 ? r.q4 : r.q6;
-        if (!((keep4 ? r.D4 : r.D6) > 0.0f)) q = 0u;          // a zero step stores +0 codes
+    const long long wg = (long long)blockIdx.x * kMqWarps + (threadIdx.x >> 5);
+    const long long nw = (long long)gridDim.x * kMqWarps;
+    const long long nblocks = (long long)a.M * (a.N / 16);
+    for (long long b0 = wg * 32; b0 < nblocks; b0 += nw * 32) {
+        const long long b = b0 + lane;
+        const bool valid = b < nblocks;
+        uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
         if (valid) {
-            a.codes[e0 / 8] = q;
-            if (!odd) a.scales[e0 / 16] = (uint8_t)(keep4 ? r.sb4 : r.sb6);
+            w0 = ld_hint(a.X + 2 * b, release);
+            w1 = ld_hint(a.X + 2 * b + 1, release);
+        }
+        float2 x[8];
+        load_x(w0, x);
+        load_x(w1, x + 4);
+        const float ab = fmaxf(max_abs8(x), max_abs8(x + 4));
+        const BlockCodes16 bc = encode_block16(x, ab, sh.tab, c, a.one);
+        if (valid) {
+            *reinterpret_cast<uint2*>(a.codes + 2 * b) = bc.q;
+            a.scales[b] = (uint8_t)bc.sb;
         }
     }
 }
