@@ -54,7 +54,7 @@ NCU_TRAFFIC = {
     "attention": ("sink_window_video_b200/csrc/attention_ws.cu",
                   "9b32bdc98dc3116b0a96d8fe5309c1a00aabf18bc35389e901e98f84d158d67b", 226354688),
     "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
-                  "90fd7b6da444df0d29b91c456b05dee9f3a7c74f6e87ceb8a00e266255452b67", 43388160),
+                  "3286f4378a02393756ca9d2ec0164e9ec70777adf69cdacefd0d340704548b10", 43654912),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
                  "ffba28cf4e3a2bc13d72d317f9f51162afdaa58cb295fff9792e1e3d0661758e", 98012416),
     "attention_fp4": ("sink_window_video_b200/csrc/attention_fp4.cu",
