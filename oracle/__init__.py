@@ -67,6 +67,7 @@ def lib():
         L.oracle_quantize_matrix.restype = i32
         L.oracle_quantize_matrix.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
         L.oracle_dequantize_matrix.argtypes = [vp, vp, f32, i32, i32, i32, vp]
+        L.oracle_rope.argtypes = [vp, i32, i32, i32, ctypes.c_int64, i32, i32, vp]
         L.oracle_set_threads.argtypes = [i32]
         L.oracle_get_threads.restype = i32
         _lib = L
@@ -287,3 +288,25 @@ def attention_f64_fp4q(chunks, Q: np.ndarray, rows=None, scale: float = 0.0) -> 
     (quantize_queries): the reference for an FP4-operand Q K^T over the cache."""
     _, Qh = quantize_queries(Q)
     return attention_f64_fq(chunks, Qh, rows, scale)
+
+
+def rope(X: np.ndarray, frame_pos0: int, rows: int, cols: int) -> np.ndarray:
+    """3D rotary position embedding of one chunk's queries or keys, X [T, H, d]
+    bf16 bits -> bf16 bits (oracle_rope in oracle.c states the reading: the
+    txtmix page "LongLive 2.0：给长视频生成补上 NVFP4 并行基础设施", sections
+    NVFP4 and 多 shot 一致性, names a fused RoPE kernel and the multi-shot RoPE
+    offset but not the rotary form).  Token t of the chunk sits at frame
+    frame_pos0 + t // (rows*cols), row (t // cols) % rows, column t % cols."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    T, H, d = X.shape
+    Y = np.empty_like(X)
+    lib().oracle_rope(_ptr(X), T, H, d, int(frame_pos0), rows, cols, _ptr(Y))
+    return Y
+
+
+def rope_frame_position(chunk: int, frames_per_chunk: int, shot: int, offset: int) -> int:
+    """Frame coordinate of chunk `chunk`'s first frame in a multi-shot stream:
+    the frames before it, plus multi_shot_rope_offset once per shot switch
+    before it (`shot` switches; the txtmix page, 多 shot 一致性: the offset keeps
+    the positions of different shots apart).  offset 0 is plain frame counting."""
+    return chunk * frames_per_chunk + shot * offset

@@ -561,6 +561,70 @@ void oracle_attention_f64_fq(const oracle_chunk* chunks, int n_chunks, int H, in
     attention_core(chunks, n_chunks, H, d, NULL, Qf, T_q, rows, n_rows, scale, out);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Rotary position embedding of a chunk's queries or keys (a reading)       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [TX] "LongLive 2.0：给长视频生成补上 NVFP4 并行基础设施" (txtmix): the section
+ * NVFP4：一条从训练贯穿到 KV cache 的量化线 names a fused RoPE kernel on the
+ * NVFP4 inference path, and 多 shot 一致性 names the inference option
+ * multi_shot_rope_offset, a RoPE position offset for multi-shot generation that
+ * keeps the positions of different shots apart.  Neither gives the rotary form.
+ * The reading taken (parity against the pages is unpinned; the tests pin this
+ * function to the properties of a rotation and to closed-form values):
+ *   - the latent tokens of a chunk form frames of rows x cols tokens, frame-major,
+ *     then row, then column: token t is at frame t / (rows*cols), row
+ *     (t / cols) % rows, column t % cols;
+ *   - the d channels of a head split into three contiguous parts, one per axis:
+ *     frame w0 = d - 4*(d/6) channels, row w1 = 2*(d/6), column w2 = 2*(d/6)
+ *     (44, 42, 42 for d = 128);
+ *   - in a part of width w, channels (2i, 2i+1) turn by the angle
+ *     p * 10000^(-2i/w), p the token's coordinate on that part's axis:
+ *     (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos);
+ *   - the frame coordinate is frame_pos0 + the frame within the chunk; a
+ *     multi-shot stream gives chunk n of shot s (s shot switches before it)
+ *     frame_pos0 = n * frames_per_chunk + s * offset, offset being
+ *     multi_shot_rope_offset (0: plain frame counting);
+ *   - arithmetic: the frequency, the angle, cos and sin in double precision;
+ *     cos and sin each rounded once to fp32; each of the four products and the
+ *     two sums one fp32 rounding; the two results rounded to bf16 (the model's
+ *     queries and keys are bf16).
+ * Y may be X (each channel pair is read before it is written).
+ */
+static void rope_cos_sin(int64_t p, int i, int w, float* c, float* s) {
+    const double omega = pow(10000.0, (double)(-2 * i) / (double)w);
+    const double phi = (double)p * omega;
+    *c = (float)cos(phi);
+    *s = (float)sin(phi);
+}
+
+void oracle_rope(const uint16_t* X, int T, int H, int d, int64_t frame_pos0, int rows,
+                 int cols, uint16_t* Y) {
+    const int w[3] = {d - 4 * (d / 6), 2 * (d / 6), 2 * (d / 6)};
+    for (int t = 0; t < T; ++t) {
+        const int64_t pos[3] = {frame_pos0 + t / (rows * cols), (t / cols) % rows, t % cols};
+        for (int h = 0; h < H; ++h) {
+            const uint16_t* x = X + ((size_t)t * H + h) * d;
+            uint16_t* y = Y + ((size_t)t * H + h) * d;
+            int base = 0;
+            for (int a = 0; a < 3; ++a) {
+                for (int i = 0; i < w[a] / 2; ++i) {
+                    float c, s;
+                    rope_cos_sin(pos[a], i, w[a], &c, &s);
+                    const float x0 = oracle_bf16_to_f32(x[base + 2 * i]);
+                    const float x1 = oracle_bf16_to_f32(x[base + 2 * i + 1]);
+                    const float x0c = x0 * c, x1s = x1 * s;
+                    const float x0s = x0 * s, x1c = x1 * c;
+                    y[base + 2 * i] = oracle_f32_to_bf16(x0c - x1s);
+                    y[base + 2 * i + 1] = oracle_f32_to_bf16(x0s + x1c);
+                }
+                base += w[a];
+            }
+        }
+    }
+}
+
 void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
 int oracle_get_threads(void) { return omp_get_max_threads(); }
 
