@@ -175,6 +175,75 @@ nvfp4kv_status nvfp4kv_quantize_chunk_noalloc(const void* K, const void* V, int 
                                               int d, const nvfp4kv_chunk_view* out,
                                               nvfp4kv_stream_t stream);
 
+/* ------------------------------------------------------------------ rotary position embedding */
+
+/*
+ * 3D rotary position embedding of a chunk's queries and keys, with the
+ * multi-shot frame offset.  Source: the txtmix page "LongLive 2.0：给长视频生成
+ * 补上 NVFP4 并行基础设施", section NVFP4：一条从训练贯穿到 KV cache 的量化线 (a
+ * fused RoPE kernel on the NVFP4 inference path), section 多 shot 一致性
+ * (inference.multi_shot_rope_offset, the RoPE position offset that keeps the
+ * positions of different shots apart).  The pages give no rotary form; the
+ * library implements this reading, whose parity with the pages is unpinned:
+ *   - token t of a chunk lies at frame t / (rows*cols), row (t / cols) % rows,
+ *     column t % cols of the latent token grid (frame-major);
+ *   - the d = 128 channels of a head split into a frame part (channels
+ *     0..43), a row part (44..85) and a column part (86..127); in a part of
+ *     width w the channel pair (2i, 2i+1) turns by the angle
+ *     p * 10000^(-2i/w), p the token's coordinate on that part's axis:
+ *     (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos);
+ *   - the frame coordinate is frame_pos0 + the frame within the chunk
+ *     (nvfp4kv_rope_frame_position gives frame_pos0 in a multi-shot stream);
+ *   - arithmetic: frequency, angle, cos and sin in double precision, cos and
+ *     sin each rounded once to fp32 (nvfp4kv_rope_table); each product and
+ *     sum of the rotation one fp32 rounding; results rounded to bf16.
+ */
+
+/* The geometry of one chunk's rotation. */
+typedef struct {
+    const void* table;   /* device, 16-byte aligned, filled by nvfp4kv_rope_table */
+    int frames;          /* frames the table covers: frames * rows * cols >= T */
+    int rows, cols;      /* latent tokens per frame: rows x cols */
+} nvfp4kv_rope_view;
+
+/* frame_pos0 of chunk `chunk` of a multi-shot stream: chunk * frames_per_chunk
+ * frames before it, plus `offset` (multi_shot_rope_offset) once for each of
+ * the `shot` shot switches before it; offset 0 counts frames as one shot.
+ * Returns -1 for a negative argument or frames_per_chunk < 1.  Host only. */
+long long nvfp4kv_rope_frame_position(long long chunk, int frames_per_chunk, long long shot,
+                                      long long offset);
+
+/* Bytes of a rotation table: 8 * (frames*22 + (rows + cols)*21), 0 for a
+ * size outside 1 <= frames <= 2^20, rows, cols >= 1 and rows*cols <= 65535. */
+size_t nvfp4kv_rope_table_bytes(int frames, int rows, int cols);
+
+/* Fill `table` (device, 16-byte aligned, nvfp4kv_rope_table_bytes long) on
+ * `stream` with float2 entries {cos, sin}: entry f*22 + i is pair i of the
+ * frame part at frame coordinate frame_pos0 + f; then rows*21 entries (row r,
+ * pair i at r*21 + i) and cols*21 entries (column c).  frame_pos0 in
+ * [0, 2^40].  One launch. */
+nvfp4kv_status nvfp4kv_rope_table(long long frame_pos0, int frames, int rows, int cols,
+                                  void* table, nvfp4kv_stream_t stream);
+
+/* Rotate X ([T][H][d] bf16, device) into Y (same layout; Y == X rotates in
+ * place, other overlaps are not allowed): the queries of a chunk whose keys go
+ * through nvfp4kv_quantize_chunk_rope with the same table.  T <= 65535,
+ * T*H*H < 2^32, frames*rows*cols >= T, and the table small enough to stage in
+ * shared memory: 8 * (27*frames + 26*(rows + cols)) <= 61440 bytes
+ * (NVFP4KV_ERR_INVALID_ARG otherwise).  One launch; bound by HBM (2 bytes
+ * read and 2 written per element). */
+nvfp4kv_status nvfp4kv_rope(const void* X, void* Y, int T, int H, int d,
+                            const nvfp4kv_rope_view* rope, nvfp4kv_stream_t stream);
+
+/* nvfp4kv_quantize_chunk of (K rotated by `rope`, V): the rotation is fused
+ * into the quantizer's two reads of K, so the rotated K is never stored; the
+ * outputs are those of nvfp4kv_quantize_chunk on nvfp4kv_rope(K), bit for
+ * bit.  The view's limits are nvfp4kv_rope's, with T = T_c. */
+nvfp4kv_status nvfp4kv_quantize_chunk_rope(const void* K, const void* V, int T_c, int H,
+                                           int d, const nvfp4kv_rope_view* rope,
+                                           const nvfp4kv_chunk_view* out, void* ws,
+                                           nvfp4kv_stream_t stream);
+
 /* ------------------------------------------------------------------ sequence parallel */
 
 /*
@@ -425,6 +494,12 @@ void kvcache_destroy(kvcache* cache);
  */
 nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const void* V,
                               nvfp4kv_stream_t stream);
+
+/* kvcache_append with K rotated by `rope` (nvfp4kv_quantize_chunk_rope): the
+ * cache holds the quantized rotated keys.  The table covers the chunk's
+ * frames (frame_pos0 = nvfp4kv_rope_frame_position of this chunk). */
+nvfp4kv_status kvcache_append_rope(kvcache* cache, int layer, const void* K, const void* V,
+                                   const nvfp4kv_rope_view* rope, nvfp4kv_stream_t stream);
 
 /*
  * Prompt switch p_k -> p_k' (DeepRead page, Method > 算法层设计): the shot

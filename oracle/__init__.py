@@ -68,6 +68,7 @@ def lib():
         L.oracle_quantize_matrix.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
         L.oracle_dequantize_matrix.argtypes = [vp, vp, f32, i32, i32, i32, vp]
         L.oracle_rope.argtypes = [vp, i32, i32, i32, ctypes.c_int64, i32, i32, vp]
+        L.oracle_rope_cos_sin.argtypes = [ctypes.c_int64, i32, i32, vp, vp]
         L.oracle_set_threads.argtypes = [i32]
         L.oracle_get_threads.restype = i32
         _lib = L
@@ -302,6 +303,15 @@ def rope(X: np.ndarray, frame_pos0: int, rows: int, cols: int) -> np.ndarray:
     Y = np.empty_like(X)
     lib().oracle_rope(_ptr(X), T, H, d, int(frame_pos0), rows, cols, _ptr(Y))
     return Y
+
+
+def rope_cos_sin(p: int, i: int, w: int):
+    """(cos, sin) of pair i's angle p * 10000^(-2i/w), each rounded once from
+    double to fp32 (the values oracle_rope turns that pair by), as float32."""
+    c = np.zeros(1, np.float32)
+    s = np.zeros(1, np.float32)
+    lib().oracle_rope_cos_sin(int(p), int(i), int(w), _ptr(c), _ptr(s))
+    return c[0], s[0]
 
 
 def rope_frame_position(chunk: int, frames_per_chunk: int, shot: int, offset: int) -> int:

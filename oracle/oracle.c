@@ -592,7 +592,7 @@ void oracle_attention_f64_fq(const oracle_chunk* chunks, int n_chunks, int H, in
  *     queries and keys are bf16).
  * Y may be X (each channel pair is read before it is written).
  */
-static void rope_cos_sin(int64_t p, int i, int w, float* c, float* s) {
+void oracle_rope_cos_sin(int64_t p, int i, int w, float* c, float* s) {
     const double omega = pow(10000.0, (double)(-2 * i) / (double)w);
     const double phi = (double)p * omega;
     *c = (float)cos(phi);
@@ -611,7 +611,7 @@ void oracle_rope(const uint16_t* X, int T, int H, int d, int64_t frame_pos0, int
             for (int a = 0; a < 3; ++a) {
                 for (int i = 0; i < w[a] / 2; ++i) {
                     float c, s;
-                    rope_cos_sin(pos[a], i, w[a], &c, &s);
+                    oracle_rope_cos_sin(pos[a], i, w[a], &c, &s);
                     const float x0 = oracle_bf16_to_f32(x[base + 2 * i]);
                     const float x1 = oracle_bf16_to_f32(x[base + 2 * i + 1]);
                     const float x0c = x0 * c, x1s = x1 * s;

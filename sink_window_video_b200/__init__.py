@@ -39,6 +39,12 @@ class ChunkView(ctypes.Structure):
                 ("k_mean", ctypes.c_void_p), ("tensor_scales", ctypes.c_void_p)]
 
 
+class RopeView(ctypes.Structure):
+    """nvfp4kv_rope_view: a chunk's rotation table (device) and token grid."""
+    _fields_ = [("table", ctypes.c_void_p), ("frames", ctypes.c_int),
+                ("rows", ctypes.c_int), ("cols", ctypes.c_int)]
+
+
 class KVCacheConfig(ctypes.Structure):
     _fields_ = [("layers", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("T_c", ctypes.c_int), ("S_g", ctypes.c_int), ("S_s", ctypes.c_int),
@@ -59,6 +65,7 @@ def load():
     st = ctypes.c_int
     cv = ctypes.POINTER(ChunkView)
     cfgp = ctypes.POINTER(KVCacheConfig)
+    rv = ctypes.POINTER(RopeView)
     sigs = {
         "nvfp4kv_chunk_bytes": (sz, [i32, i32, i32]),
         "nvfp4kv_chunk_view_init": (st, [vp, i32, i32, i32, cv]),
@@ -75,6 +82,14 @@ def load():
                                         vp]),
         "nvfp4kv_attention_fp4q_launches": (i32, [i32, i32, i32, i32, i32]),
         "nvfp4kv_matrix_workspace_bytes": (sz, []),
+        "nvfp4kv_rope_frame_position": (ctypes.c_longlong, [ctypes.c_longlong, i32,
+                                                            ctypes.c_longlong,
+                                                            ctypes.c_longlong]),
+        "nvfp4kv_rope_table_bytes": (sz, [i32, i32, i32]),
+        "nvfp4kv_rope_table": (st, [ctypes.c_longlong, i32, i32, i32, vp, vp]),
+        "nvfp4kv_rope": (st, [vp, vp, i32, i32, i32, rv, vp]),
+        "nvfp4kv_quantize_chunk_rope": (st, [vp, vp, i32, i32, i32, rv, cv, vp, vp]),
+        "kvcache_append_rope": (st, [vp, i32, vp, vp, rv, vp]),
         "nvfp4kv_chunk_stats": (st, [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
         "nvfp4kv_chunk_finalize": (st, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
         "nvfp4kv_chunk_amax": (st, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
@@ -344,6 +359,59 @@ def quantize_chunk(K, V, out: ChunkBuffer, ws, stream=None):
                                          _ptr(ws), _stream(stream)), "nvfp4kv_quantize_chunk")
 
 
+# ------------------------------------------------------------------ rotary position embedding
+
+def rope_frame_position(chunk, frames_per_chunk, shot, offset) -> int:
+    """frame_pos0 of a chunk of a multi-shot stream: chunk * frames_per_chunk
+    plus multi_shot_rope_offset once per shot switch before it."""
+    p = int(load().nvfp4kv_rope_frame_position(int(chunk), int(frames_per_chunk), int(shot),
+                                                int(offset)))
+    if p < 0:
+        raise NvFp4KvError(ERR_INVALID_ARG, "nvfp4kv_rope_frame_position")
+    return p
+
+
+class RopeTable:
+    """A chunk's rotation table on the device (nvfp4kv_rope_table) and the
+    token grid it covers: `frames` frames of rows x cols tokens."""
+
+    def __init__(self, frames, rows, cols, device="cuda"):
+        import torch
+        n = int(load().nvfp4kv_rope_table_bytes(frames, rows, cols))
+        if n == 0:
+            raise NvFp4KvError(ERR_INVALID_ARG, "nvfp4kv_rope_table_bytes")
+        self.table = torch.empty(n // 4, dtype=torch.float32, device=device)
+        self.view = RopeView(self.table.data_ptr(), frames, rows, cols)
+        self.frames, self.rows, self.cols = frames, rows, cols
+
+    def fill(self, frame_pos0, stream=None):
+        """Compute the table for a chunk whose first frame is at frame_pos0."""
+        _check(load().nvfp4kv_rope_table(int(frame_pos0), self.frames, self.rows, self.cols,
+                                         _ptr(self.table), _stream(stream)),
+               "nvfp4kv_rope_table")
+        return self
+
+
+def rope(X, table: RopeTable, Y=None, stream=None):
+    """Rotate bf16 [T, H, d] X into Y (a new tensor when None; Y = X in place)."""
+    import torch
+    T, H, d = X.shape
+    if Y is None:
+        Y = torch.empty_like(X)
+    _check(load().nvfp4kv_rope(_ptr(X), _ptr(Y), T, H, d, ctypes.byref(table.view),
+                               _stream(stream)), "nvfp4kv_rope")
+    return Y
+
+
+def quantize_chunk_rope(K, V, table: RopeTable, out: ChunkBuffer, ws, stream=None):
+    """quantize_chunk of (K rotated by `table`, V), the rotation fused."""
+    T, H, d = K.shape
+    _check(load().nvfp4kv_quantize_chunk_rope(_ptr(K), _ptr(V), T, H, d,
+                                              ctypes.byref(table.view), ctypes.byref(out.view),
+                                              _ptr(ws), _stream(stream)),
+           "nvfp4kv_quantize_chunk_rope")
+
+
 def quantize_chunk_noalloc(K, V, out: ChunkBuffer, stream=None):
     """quantize_chunk without a workspace: the library's compiled-in scratch
     (chunks whose scratch exceeds it are refused with ERR_CAPACITY)."""
@@ -476,6 +544,11 @@ class KVCache:
     def append(self, layer, K, V, stream=None):
         _check(load().kvcache_append(self._h, layer, _ptr(K), _ptr(V), _stream(stream)),
                "kvcache_append")
+
+    def append_rope(self, layer, K, V, table: "RopeTable", stream=None):
+        _check(load().kvcache_append_rope(self._h, layer, _ptr(K), _ptr(V),
+                                          ctypes.byref(table.view), _stream(stream)),
+               "kvcache_append_rope")
 
     def advance(self, layer):
         v = ChunkView()

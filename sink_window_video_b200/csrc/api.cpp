@@ -121,6 +121,33 @@ bool have_sm100() {
     return state == 1;
 }
 
+// A rotation's grid: every size at least 1, rows*cols < 2^16 and at most
+// 2^20 frames (the table's index and the token division stay in 32 bits).
+bool rope_grid_ok(int frames, int rows, int cols) {
+    return frames >= 1 && rows >= 1 && cols >= 1 && frames <= (1 << 20) &&
+           (long long)rows * cols <= 65535;
+}
+
+// The rotation of T tokens: a valid view whose table covers them and fits the
+// consumers' shared memory when staged.
+nvfp4kv_status check_rope_view(const nvfp4kv_rope_view* r, int T) {
+    if (!r || !r->table || !rope_grid_ok(r->frames, r->rows, r->cols) || T > 65535 ||
+        (long long)r->frames * r->rows * r->cols < T ||
+        nvfp4kv::rope_staged_bytes(r->frames, r->rows, r->cols) > nvfp4kv::kRopeMaxStagedBytes)
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (!aligned16(r->table)) return NVFP4KV_ERR_ALIGNMENT;
+    return NVFP4KV_OK;
+}
+
+nvfp4kv::RopeGeom rope_geom(const nvfp4kv_rope_view& r) {
+    nvfp4kv::RopeGeom g;
+    g.table = r.table;
+    g.frames = r.frames;
+    g.rows = r.rows;
+    g.cols = r.cols;
+    return g;
+}
+
 }  // namespace
 
 namespace nvfp4kv {
@@ -202,6 +229,51 @@ nvfp4kv_status nvfp4kv_quantize_chunk(const void* K, const void* V, int T_c, int
     const nvfp4kv_status st = check_quantize_chunk_args(K, V, T_c, H, d, out, ws, true);
     if (st != NVFP4KV_OK) return st;
     return launch_quantize(K, V, T_c, H, *out, ws, (cudaStream_t)stream);
+}
+
+long long nvfp4kv_rope_frame_position(long long chunk, int frames_per_chunk, long long shot,
+                                      long long offset) {
+    if (chunk < 0 || frames_per_chunk < 1 || shot < 0 || offset < 0) return -1;
+    return chunk * frames_per_chunk + shot * offset;
+}
+
+size_t nvfp4kv_rope_table_bytes(int frames, int rows, int cols) {
+    if (!rope_grid_ok(frames, rows, cols)) return 0;
+    return 8 * rope_table_entries(frames, rows, cols);
+}
+
+nvfp4kv_status nvfp4kv_rope_table(long long frame_pos0, int frames, int rows, int cols,
+                                  void* table, nvfp4kv_stream_t stream) {
+    if (!table || !rope_grid_ok(frames, rows, cols) || frame_pos0 < 0 ||
+        frame_pos0 > (1LL << 40))
+        return NVFP4KV_ERR_INVALID_ARG;
+    if (!aligned16(table)) return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_rope_table(frame_pos0, frames, rows, cols, table, (cudaStream_t)stream);
+}
+
+nvfp4kv_status nvfp4kv_rope(const void* X, void* Y, int T, int H, int d,
+                            const nvfp4kv_rope_view* rope, nvfp4kv_stream_t stream) {
+    if (!X || !Y || !valid_shape(T, H, d) || (long long)T * H * H >= (1LL << 32))
+        return NVFP4KV_ERR_INVALID_ARG;
+    const nvfp4kv_status st = check_rope_view(rope, T);
+    if (st != NVFP4KV_OK) return st;
+    if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
+    if (!aligned16(X) || !aligned16(Y)) return NVFP4KV_ERR_ALIGNMENT;
+    if (!have_sm100()) return NVFP4KV_ERR_UNSUPPORTED;
+    return launch_rope(X, Y, T, H, rope_geom(*rope), (cudaStream_t)stream);
+}
+
+nvfp4kv_status nvfp4kv_quantize_chunk_rope(const void* K, const void* V, int T_c, int H,
+                                           int d, const nvfp4kv_rope_view* rope,
+                                           const nvfp4kv_chunk_view* out, void* ws,
+                                           nvfp4kv_stream_t stream) {
+    nvfp4kv_status st = check_rope_view(rope, T_c);
+    if (st != NVFP4KV_OK) return st;
+    st = check_quantize_chunk_args(K, V, T_c, H, d, out, ws, true);
+    if (st != NVFP4KV_OK) return st;
+    const RopeGeom g = rope_geom(*rope);
+    return launch_quantize(K, V, T_c, H, *out, ws, (cudaStream_t)stream, &g);
 }
 
 nvfp4kv_status nvfp4kv_chunk_stats(const void* K, const void* V, int T_local, int H, int d,
@@ -515,9 +587,14 @@ nvfp4kv_status kvcache_set_state(kvcache* cache, const void* buf, size_t bytes) 
     return NVFP4KV_OK;
 }
 
-nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const void* V,
-                              nvfp4kv_stream_t stream) {
+namespace {
+nvfp4kv_status cache_append(kvcache* cache, int layer, const void* K, const void* V,
+                            const nvfp4kv_rope_view* rope, nvfp4kv_stream_t stream) {
     if (!cache || !K || !V) return NVFP4KV_ERR_INVALID_ARG;
+    if (rope) {
+        const nvfp4kv_status r = check_rope_view(rope, cache->cfg.T_c);
+        if (r != NVFP4KV_OK) return r;
+    }
     if (layer < 0 || layer >= cache->cfg.layers) return NVFP4KV_ERR_CAPACITY;
     if (cache->cfg.d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;
     if (!aligned16(K) || !aligned16(V)) return NVFP4KV_ERR_ALIGNMENT;
@@ -530,8 +607,24 @@ nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const vo
     nvfp4kv_chunk_view v;
     nvfp4kv_status st = kvcache_advance(cache, layer, &v);
     if (st != NVFP4KV_OK || v.k_codes == nullptr) return st;
+    if (!rope)
+        return launch_quantize(K, V, cache->cfg.T_c, cache->cfg.H, v, cache->ws,
+                               (cudaStream_t)stream);
+    const RopeGeom g = rope_geom(*rope);
     return launch_quantize(K, V, cache->cfg.T_c, cache->cfg.H, v, cache->ws,
-                           (cudaStream_t)stream);
+                           (cudaStream_t)stream, &g);
+}
+}  // namespace
+
+nvfp4kv_status kvcache_append(kvcache* cache, int layer, const void* K, const void* V,
+                              nvfp4kv_stream_t stream) {
+    return cache_append(cache, layer, K, V, nullptr, stream);
+}
+
+nvfp4kv_status kvcache_append_rope(kvcache* cache, int layer, const void* K, const void* V,
+                                   const nvfp4kv_rope_view* rope, nvfp4kv_stream_t stream) {
+    if (!rope) return NVFP4KV_ERR_INVALID_ARG;
+    return cache_append(cache, layer, K, V, rope, stream);
 }
 
 nvfp4kv_status sink_window_attention(const kvcache* cache, int layer, const void* Q, int T_q,

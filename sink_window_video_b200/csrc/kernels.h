@@ -92,8 +92,11 @@ nvfp4kv_status check_quantize_chunk_args(const void* K, const void* V, int T_c, 
                                          const nvfp4kv_chunk_view* out, const void* ws,
                                          bool need_ws);
 
+struct RopeGeom;
+// rope: K is rotated (rope.cu's reading) before it is quantized; null for none.
 nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
-                               const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream);
+                               const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream,
+                               const RopeGeom* rope = nullptr);
 
 // Sequence-parallel phases of the chunk quantizer (quant.cu).
 nvfp4kv_status launch_sp_stats(const void* K, const void* V, int T_local, int H, float* psum,
@@ -115,6 +118,22 @@ size_t matrix_workspace_bytes();
 nvfp4kv_status launch_quantize_matrix(const void* X, int M, int N, int mode, void* codes,
                                       void* scales, float* tensor_scale, void* ws,
                                       cudaStream_t stream);
+
+// 3D rotary position embedding (rope.cu): a chunk's cos/sin table and the
+// frame grid of its tokens (frames * rows * cols >= T).
+struct RopeGeom {
+    const void* table;
+    int frames, rows, cols;
+};
+size_t rope_table_entries(int frames, int rows, int cols);
+// Shared memory of a staged table (rope.cuh's padded rows); kernels that stage
+// it take grids up to kRopeMaxStagedBytes.
+constexpr size_t kRopeMaxStagedBytes = 61440;
+size_t rope_staged_bytes(int frames, int rows, int cols);
+nvfp4kv_status launch_rope_table(long long frame_pos0, int frames, int rows, int cols,
+                                 void* table, cudaStream_t stream);
+nvfp4kv_status launch_rope(const void* X, void* Y, int T, int H, const RopeGeom& r,
+                           cudaStream_t stream);
 
 int sm_count_cached();
 nvfp4kv_status launch_dequantize(const nvfp4kv_chunk_view& in, int T, int H, void* K_out,

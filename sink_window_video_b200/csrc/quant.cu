@@ -42,6 +42,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "nvfp4_encode.cuh"
+#include "rope.cuh"
 
 namespace nvfp4kv {
 namespace {
@@ -73,6 +74,7 @@ struct QuantArgs {
     float* vpart;
     Control* ctl;
     float one;              // 1 as a run-time value (see encode8_fast)
+    RopeDev rope;           // quantize_kernel<true>: K is rotated first (rope.cu)
 };
 
 // Shared memory of the chunk quantizer (the sequence-parallel kernels use the
@@ -247,8 +249,19 @@ __device__ __forceinline__ void stats_k_token(const uint4& w, float* sum, uint32
     }
 }
 
-// One (64-token segment, 256-column group) of K: lane = 8 columns.
-__device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
+// K rotated (rope.cu's reading): the 8 channels of w, head pair group q, of
+// token t, with the table staged in shared memory (rsm).
+__device__ __forceinline__ uint4 rope_k8(const RopeDev& g, const float2* rsm, const RopeGroup& q,
+                                         uint4 w, int t) {
+    uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    rope_group4(q, rope_rows(g, (uint32_t)t), rsm, g.one, u);
+    return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+// One (64-token segment, 256-column group) of K: lane = 8 columns (with ROPE,
+// of the rotated K).
+template <bool ROPE>
+__device__ void stats_unit(const QuantArgs& a, const float2* rsm, int unit, uint64_t keep) {
     const int lane = threadIdx.x & 31;
     const int s = unit / a.ngroups;
     const int g = unit - s * a.ngroups;
@@ -264,15 +277,23 @@ __device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
     for (int i = 0; i < 8; ++i) sum[i] = 0.0f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) { mn[j] = 0x7F807F80u; mx[j] = 0xFF80FF80u; }
+    const RopeGroup grp = rope_group((lane & 15) * 4);   // the lane's four head pairs
     int t = 0;
     for (; t + kStatsBatch <= nt; t += kStatsBatch) {
         uint4 w[kStatsBatch];
 #pragma unroll
         for (int k = 0; k < kStatsBatch; ++k) w[k] = ld_hint(src + (size_t)(t + k) * row8, keep);
 #pragma unroll
-        for (int k = 0; k < kStatsBatch; ++k) stats_k_token(w[k], sum, mn, mx);
+        for (int k = 0; k < kStatsBatch; ++k) {
+            if (ROPE) w[k] = rope_k8(a.rope, rsm, grp, w[k], t0 + t + k);
+            stats_k_token(w[k], sum, mn, mx);
+        }
     }
-    for (; t < nt; ++t) stats_k_token(ld_hint(src + (size_t)t * row8, keep), sum, mn, mx);
+    for (; t < nt; ++t) {
+        uint4 w = ld_hint(src + (size_t)t * row8, keep);
+        if (ROPE) w = rope_k8(a.rope, rsm, grp, w, t0 + t);
+        stats_k_token(w, sum, mn, mx);
+    }
     float4* ps = reinterpret_cast<float4*>(a.psum + (size_t)s * a.HD + col);
     ps[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
     ps[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
@@ -288,9 +309,10 @@ __device__ void stats_unit(const QuantArgs& a, int unit, uint64_t keep) {
 // within a step, 16-channel block), one block per lane (encode_block16);
 // step it covers tokens t0 + 4 it + {0..3}, with the next step's loads in
 // flight.
-template <bool IS_K>
+template <bool IS_K, bool ROPE>
 __device__ void encode_unit(const QuantArgs& a, const float2* tab, const EncodeConsts& c,
-                            uint8_t* sbst, int h, int t0, uint64_t release) {
+                            uint8_t* sbst, int h, int t0, uint64_t release,
+                            const float2* rsm = nullptr) {
     const int lane = threadIdx.x & 31;
     const int blk = lane & 7;                 // 16-channel block of this lane
     const int tsub = lane >> 3;               // token within a step
@@ -327,7 +349,13 @@ __device__ void encode_unit(const QuantArgs& a, const float2* tab, const EncodeC
         }
         float2 x[8];
         {
-            const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            if (IS_K && ROPE && (full || 4 * it < nt)) {
+                // the rotated K: head pairs 8 blk .. 8 blk + 7 of this lane's token
+                const RopeRows b = rope_rows(a.rope, (uint32_t)(t0 + tsub + 4 * it));
+                rope_group4(rope_group(8 * blk), b, rsm, a.rope.one, u);
+                rope_group4(rope_group(8 * blk + 4), b, rsm, a.rope.one, u + 4);
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 // bf16 -> fp32 exactly (signed zeros kept)
@@ -488,8 +516,11 @@ __device__ __forceinline__ int take(unsigned* q, int n, volatile int* abort) {
     return i < n ? i : -1;
 }
 
+template <bool ROPE>
 __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a) {
     __shared__ QuantShared sh;
+    extern __shared__ float2 rope_sm[];           // ROPE: the staged rotation table
+    if (ROPE) rope_stage(a.rope, rope_sm);        // published by phase_vmax's barriers
     const uint64_t keep = policy_keep(), release = policy_release();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -521,7 +552,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
     if (warp < kStatsWarps) {
         // 2a. K statistics from HBM
         int done = 0;
-        for (int i; (i = take(&sh.q_stats, s1 - s0, abort)) >= 0; ++done) stats_unit(a, s0 + i, keep);
+        for (int i; (i = take(&sh.q_stats, s1 - s0, abort)) >= 0; ++done)
+            stats_unit<ROPE>(a, rope_sm, s0 + i, keep);
         __threadfence();
         if (lane == 0 && done > 0) atomicAdd(&a.ctl->q_sdone, (unsigned)done);
         // 2b. this CTA's column blocks, once every CTA's statistics are in
@@ -549,7 +581,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
         for (int i; (i = take(&sh.q_v, u1 - u0, abort)) >= 0;) {
             const int u = u0 + i;
             const int h = u / tiles;
-            encode_unit<false>(a, sh.tab[0], c, sbst, h, (u - h * tiles) * kEncTokens, release);
+            encode_unit<false, false>(a, sh.tab[0], c, sbst, h, (u - h * tiles) * kEncTokens,
+                                      release);
         }
     }
     // 3. K from L2
@@ -559,7 +592,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
         for (int i; (i = take(&sh.q_k, u1 - u0, abort)) >= 0;) {
             const int u = u0 + i;
             const int h = u / tiles;
-            encode_unit<true>(a, sh.tab[1], c, sbst, h, (u - h * tiles) * kEncTokens, release);
+            encode_unit<true, ROPE>(a, sh.tab[1], c, sbst, h, (u - h * tiles) * kEncTokens,
+                                    release, rope_sm);
         }
     }
     __syncthreads();
@@ -602,7 +636,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) sp_stats_kernel(QuantArgs a,
     const uint64_t keep = policy_keep();
     const int wg = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     const int nw = gridDim.x * kQuantWarps;
-    for (int u = wg; u < a.nseg * a.ngroups; u += nw) stats_unit(a, u, keep);
+    for (int u = wg; u < a.nseg * a.ngroups; u += nw) stats_unit<false>(a, nullptr, u, keep);
     const float b = phase_vmax(a, sh, keep);         // per-CTA max |V| ...
     if (threadIdx.x == 0) atomicMax(vmax_bits, __float_as_uint(b));
 }
@@ -656,9 +690,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1) sp_encode_kernel(QuantArgs a
         const int h = u / tiles;
         const int t0 = (u - h * tiles) * kEncTokens;
         if (isK)
-            encode_unit<true>(a, sh.tab[0], c, sh.sb[warp], h, t0, release);
+            encode_unit<true, false>(a, sh.tab[0], c, sh.sb[warp], h, t0, release);
         else
-            encode_unit<false>(a, sh.tab[0], c, sh.sb[warp], h, t0, release);
+            encode_unit<false, false>(a, sh.tab[0], c, sh.sb[warp], h, t0, release);
     }
 }
 
@@ -699,22 +733,30 @@ __global__ void check_formats_kernel(int op, const float* fin, const uint8_t* bi
     }
 }
 
-int g_quant_grid[64];   // cooperative grid size per device ordinal (0 = not yet known)
+int g_quant_grid[2][64];   // cooperative grid size per kernel and device ordinal (0: unknown)
 
 }  // namespace
 
 nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
-                               const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream) {
+                               const nvfp4kv_chunk_view& out, void* ws, cudaStream_t stream,
+                               const RopeGeom* rope) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4KV_ERR_CUDA;
-    if (g_quant_grid[dev] == 0) {
+    const void* kernel = rope ? (const void*)quantize_kernel<true> : (const void*)quantize_kernel<false>;
+    int& grid = g_quant_grid[rope ? 1 : 0][dev];
+    if (grid == 0) {
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return NVFP4KV_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel, kQuantThreads,
-                                                          0) != cudaSuccess || per_sm < 1)
+        const size_t dyn = rope ? kRopeMaxStagedBytes : 0;
+        if (rope && cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)dyn) != cudaSuccess)
             return NVFP4KV_ERR_CUDA;
-        g_quant_grid[dev] = min(sms * per_sm, kMaxGrid);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, dyn) !=
+                cudaSuccess ||
+            per_sm < 1)
+            return NVFP4KV_ERR_CUDA;
+        grid = min(sms * per_sm, kMaxGrid);
     }
     const WsLayout L = ws_layout(T, H);
     char* w = static_cast<char*>(ws);
@@ -739,10 +781,11 @@ nvfp4kv_status launch_quantize(const void* K, const void* V, int T, int H,
     a.vpart = reinterpret_cast<float*>(w + L.vpart);
     a.ctl = reinterpret_cast<Control*>(w);
     a.one = 1.0f;
+    a.rope = rope ? rope_dev(*rope) : RopeDev{};
     void* args[] = {&a};
-    cudaError_t e = cudaLaunchCooperativeKernel((const void*)quantize_kernel,
-                                                dim3(g_quant_grid[dev]), dim3(kQuantThreads),
-                                                args, 0, stream);
+    const size_t smem = rope ? rope_staged_bytes(rope->frames, rope->rows, rope->cols) : 0;
+    cudaError_t e = cudaLaunchCooperativeKernel(kernel, dim3(grid), dim3(kQuantThreads), args,
+                                                smem, stream);
     return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 

@@ -352,3 +352,63 @@ def test_cache_state_refusals_change_nothing(L):
     assert _set(L, h, good) == swv.OK
     L.kvcache_destroy(h)
     L.kvcache_destroy(other)
+
+
+def test_rope_entry_points_refuse_bad_arguments(L):
+    """The rotary embedding's host checks, before any device work."""
+    assert L.nvfp4kv_rope_frame_position(5, 8, 2, 1000) == 40 + 2000
+    assert L.nvfp4kv_rope_frame_position(3, 8, 0, 0) == 24
+    for bad in [(-1, 8, 0, 0), (1, 0, 0, 0), (1, 8, -1, 0), (1, 8, 0, -5)]:
+        assert L.nvfp4kv_rope_frame_position(*bad) == -1
+    assert L.nvfp4kv_rope_table_bytes(8, 22, 40) == 8 * (8 * 22 + (22 + 40) * 21)
+    for bad in [(0, 22, 40), (8, 0, 40), (8, 22, 0), (1, 256, 256), (1 << 21, 1, 1)]:
+        assert L.nvfp4kv_rope_table_bytes(*bad) == 0
+    # table
+    assert L.nvfp4kv_rope_table(0, 8, 22, 40, None, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope_table(-1, 8, 22, 40, FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope_table((1 << 40) + 1, 8, 22, 40, FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope_table(0, 0, 22, 40, FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope_table(0, 8, 22, 40, FAKE + 8, None) == swv.ERR_ALIGNMENT
+    # rotation
+    view = swv.RopeView(FAKE, 8, 22, 40)
+    r = ctypes.byref(view)
+    assert L.nvfp4kv_rope(None, FAKE, 7040, 24, 128, r, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope(FAKE, FAKE, 7040, 24, 128, None, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope(FAKE, FAKE, 7041, 24, 128, r, None) == swv.ERR_INVALID_ARG  # > 8 frames
+    assert L.nvfp4kv_rope(FAKE, FAKE, 0, 24, 128, r, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_rope(FAKE, FAKE, 7040, 24, 96, r, None) == swv.ERR_UNSUPPORTED
+    assert L.nvfp4kv_rope(FAKE + 8, FAKE, 7040, 24, 128, r, None) == swv.ERR_ALIGNMENT
+    assert L.nvfp4kv_rope(FAKE, FAKE, 100, 1 << 13, 128, r, None) == swv.ERR_INVALID_ARG
+    big = swv.RopeView(FAKE, 2, 300, 300)                       # rows * cols > 65535
+    assert L.nvfp4kv_rope(FAKE, FAKE, 100, 2, 128, ctypes.byref(big), None) == \
+        swv.ERR_INVALID_ARG
+    wide = swv.RopeView(FAKE, 1, 100, 200)                      # too large to stage
+    assert L.nvfp4kv_rope(FAKE, FAKE, 100, 2, 128, ctypes.byref(wide), None) == \
+        swv.ERR_INVALID_ARG
+    huge = swv.RopeView(FAKE, 100, 22, 40)                      # T > 65535
+    assert L.nvfp4kv_rope(FAKE, FAKE, 70000, 1, 128, ctypes.byref(huge), None) == \
+        swv.ERR_INVALID_ARG
+    for bad_view in [swv.RopeView(None, 8, 22, 40), swv.RopeView(FAKE, 0, 22, 40)]:
+        assert L.nvfp4kv_rope(FAKE, FAKE, 7040, 24, 128, ctypes.byref(bad_view), None) == \
+            swv.ERR_INVALID_ARG
+    unaligned = swv.RopeView(FAKE + 4, 8, 22, 40)
+    assert L.nvfp4kv_rope(FAKE, FAKE, 7040, 24, 128, ctypes.byref(unaligned), None) == \
+        swv.ERR_ALIGNMENT
+    # fused quantizer and cache append
+    v = swv.chunk_view_init(FAKE, 7040, 24)
+    assert L.nvfp4kv_quantize_chunk_rope(FAKE, FAKE, 7040, 24, 128, None, ctypes.byref(v),
+                                         FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_quantize_chunk_rope(FAKE, FAKE, 7041, 24, 128, r, ctypes.byref(v),
+                                         FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_quantize_chunk_rope(None, FAKE, 7040, 24, 128, r, ctypes.byref(v),
+                                         FAKE, None) == swv.ERR_INVALID_ARG
+    assert L.nvfp4kv_quantize_chunk_rope(FAKE, FAKE, 7040, 24, 128, r, ctypes.byref(v),
+                                         None, None) == swv.ERR_INVALID_ARG
+    h, _ = _cache(L, 1, 1, 1, 2, T=32, H=2)
+    small = swv.RopeView(FAKE, 1, 4, 4)                         # 16 tokens < T_c = 32
+    assert L.kvcache_append_rope(h, 0, FAKE, FAKE, None, None) == swv.ERR_INVALID_ARG
+    assert L.kvcache_append_rope(h, 0, FAKE, FAKE, ctypes.byref(small), None) == \
+        swv.ERR_INVALID_ARG
+    n = ctypes.c_int64()
+    assert L.kvcache_num_chunks(h, 0, ctypes.byref(n)) == swv.OK and n.value == 0
+    L.kvcache_destroy(h)
