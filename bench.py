@@ -59,6 +59,8 @@ NCU_TRAFFIC = {
                  "ffba28cf4e3a2bc13d72d317f9f51162afdaa58cb295fff9792e1e3d0661758e", 98012416),
     "attention_fp4": ("sink_window_video_b200/csrc/attention_fp4.cu",
                       "385b563baf2156d9f340a5b351f880de978d2ecddd7e92a3ddefc57bd36f4a2b", 194231296),
+    "rope": ("sink_window_video_b200/csrc/rope.cu",
+             "99749510966436bda09ff494d743697066680af300e7be7131e030868f696f84", 45756160),
     "dequantize": ("sink_window_video_b200/csrc/dequant.cu",
                    "7dd04c898e146642244e3c647f75a4c6d746e2fad0c7c310a2255267bb2fd8f6", 51334400),
 }
@@ -324,6 +326,7 @@ def run_ours(args, rank, world, local):
     dequant = run_dequant(swv, cache, stream) if not args.no_matrix else None
     qonly = run_quantize_only(swv, stream) if not args.no_quantize_only else None
     fp4q = run_fp4q(swv, cache, pool, O, stream) if not args.no_fp4q else None
+    rope = run_rope(swv, pool, stream) if not args.no_rope else None
 
     rollouts = None
     if not args.no_rollout:
@@ -331,7 +334,7 @@ def run_ours(args, rank, world, local):
 
     return dict(ms_total=ms_total, ms_quant=ms_quant, ms_attn=ms_attn, clocks=clocks,
                 e2e_ms=e2e_ms, rollouts=rollouts, matrix=matrix, dequant=dequant,
-                quantize_only=qonly, fp4q=fp4q,
+                quantize_only=qonly, fp4q=fp4q, rope=rope,
                 attn_launches=swv.attention_launches(len(cache.keyset(0)), T, H, T))
 
 
@@ -423,6 +426,66 @@ def run_dequant(swv, cache, stream, launches=40):
             "bytes_per_launch": nbytes, "achieved": gbs, "unit": "GB/s", "peak": hpeak,
             "frac": gbs / hpeak, "bound": "hbm", "gpu_launches_per_call": 1,
             "traffic": ncu_traffic("dequantize"), "peak_source": f"{src} hbm"}
+
+
+# ------------------------------------------------------------------ rotary position embedding
+
+ROPE_GRID = (8, 22, 40)          # frames per chunk, latent rows, latent columns: 7040 tokens
+ROPE_CHUNK = 9                   # the layer step's chunk: frames 72..79 of a single shot
+
+
+def run_rope(swv, pool, stream, launches=40):
+    """The 3D rotary embedding of the layer step's chunk: its cos/sin table, the
+    rotation of the queries [7040, 24, 128] (rotating over the pool's Q tensors,
+    larger than L2), and the chunk quantizer with the rotation fused into its
+    reads of K, beside the quantizer alone and the unfused composition (rotate,
+    then quantize).  CUDA events around each launch."""
+    import torch
+    peaks, src = load_peaks()
+    hpeak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    T, H, d = CFG["T_c"], CFG["H"], CFG["d"]
+    F, R, C = ROPE_GRID
+    tab = swv.RopeTable(F, R, C)
+    p0 = swv.rope_frame_position(ROPE_CHUNK, F, 0, 0)
+    ws = swv.new_workspace(T, H)
+    out = swv.ChunkBuffer(T, H)
+    Y = torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda")
+    n = len(pool)
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(launches)]
+        torch.cuda.synchronize()
+        for i, (e0, e1) in enumerate(ev):
+            e0.record(stream)
+            fn(i)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * sum(e0.elapsed_time(e1) for e0, e1 in ev) / launches
+
+    t_table = timed(lambda i: tab.fill(p0))
+    t_rope = timed(lambda i: swv.rope(pool[i % n][2], tab, Y=Y))
+    t_q = timed(lambda i: swv.quantize_chunk(pool[i % n][0], pool[i % n][1], out, ws))
+    t_qr = timed(lambda i: swv.quantize_chunk_rope(pool[i % n][0], pool[i % n][1], tab, out, ws))
+    if swv.workspace_status(ws) != swv.OK:
+        raise RuntimeError("device status not OK after the rotary quantizer")
+    rb = 4 * T * H * d                         # bf16 in and out
+    qb = quant_bytes()
+    return {"workload": f"chunk {ROPE_CHUNK} of a single shot: {F} frames of {R} x {C} tokens, "
+                        f"frame coordinates {p0}..{p0 + F - 1}",
+            "table_us": t_table,
+            "rope": {"kernel": "nvfp4kv_rope (queries [7040, 24, 128] bf16)", "us_per_launch": t_rope,
+                     "bytes_per_launch": rb, "achieved": rb / (t_rope / 1e6) / 1e9, "unit": "GB/s",
+                     "peak": hpeak, "frac": rb / (t_rope / 1e6) / 1e9 / hpeak, "bound": "hbm",
+                     "traffic": ncu_traffic("rope"), "peak_source": f"{src} hbm"},
+            "quantize_rope": {"kernel": "nvfp4kv_quantize_chunk_rope (rotation fused)",
+                              "us_per_launch": t_qr, "bytes_per_launch": qb,
+                              "achieved": qb / (t_qr / 1e6) / 1e9, "unit": "GB/s", "peak": hpeak,
+                              "frac": qb / (t_qr / 1e6) / 1e9 / hpeak, "bound": "hbm",
+                              "peak_source": f"{src} hbm",
+                              "quantize_alone_us": t_q, "unfused_us": t_rope + t_q}}
 
 
 # ------------------------------------------------------------------ FP4-operand attention
@@ -782,6 +845,8 @@ def build_line(args, r, world, peaks, peak_src):
         line["quantize_only"] = r["quantize_only"]
     if r.get("fp4q") is not None:
         line["attention_fp4q"] = r["fp4q"]
+    if r.get("rope") is not None:
+        line["rope"] = r["rope"]
     return line
 
 
@@ -798,6 +863,7 @@ def main():
     ap.add_argument("--no-matrix", action="store_true")
     ap.add_argument("--no-quantize-only", action="store_true")
     ap.add_argument("--no-fp4q", action="store_true")
+    ap.add_argument("--no-rope", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
     args = ap.parse_args()
     if args.warmup < 3:

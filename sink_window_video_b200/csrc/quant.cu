@@ -50,12 +50,13 @@ namespace {
 constexpr int kQuantThreads = 768;       // one CTA per SM: 24 warps
 constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kStatsWarps = 10;          // warps 0-9 read K's statistics first
+constexpr int kStatsWarpsRope = 15;      // with K rotated: its statistics cost ~3x
 constexpr int kEncTokens = 16;           // tokens per encoding unit (one warp)
 constexpr int kFinCols = 32;             // columns per finalize block (one per lane)
 constexpr int kStatsBatch = 8;           // K rows in flight per lane in the statistics pass
 constexpr int kFinSegs = 120;            // segments staged per finalize pass
-constexpr int kSegsPerStatsWarp = kFinSegs / kStatsWarps;
-static_assert(kFinSegs % kStatsWarps == 0, "finalize staging splits evenly");
+static_assert(kFinSegs % kStatsWarps == 0 && kFinSegs % kStatsWarpsRope == 0,
+              "finalize staging splits evenly");
 
 struct QuantArgs {
     const uint4* K;
@@ -389,10 +390,12 @@ __device__ void encode_unit(const QuantArgs& a, const float2* tab, const EncodeC
 // ---------------------------------------------------------------- finalize
 
 // The mean and max |K - mean| of a 32-column block from every segment's
-// statistics: the statistics warps (256 threads, named barrier 1) stage the
-// segments in shared memory, warp 0 adds them in segment order.  Returns
+// statistics: the NSW statistics warps (named barrier 1) stage the segments in
+// shared memory, warp 0 adds them in segment order.  Returns
 // (in warp 0) the block's max |K - mean|.
+template <int NSW>
 __device__ float finalize_block(const QuantArgs& a, QuantShared& sh, int b) {
+    constexpr int kSegsPerStatsWarp = kFinSegs / NSW;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int col = b * kFinCols + lane;
@@ -405,7 +408,7 @@ __device__ float finalize_block(const QuantArgs& a, QuantShared& sh, int b) {
         unsigned short pn[kSegsPerStatsWarp], px[kSegsPerStatsWarp];
 #pragma unroll
         for (int j = 0; j < kSegsPerStatsWarp; ++j) {
-            const int k = warp + j * kStatsWarps;
+            const int k = warp + j * NSW;
             if (k < ns) {
                 const size_t i = (size_t)(s0 + k) * a.HD + col;
                 ps[j] = __ldcg(a.psum + i);
@@ -415,14 +418,14 @@ __device__ float finalize_block(const QuantArgs& a, QuantShared& sh, int b) {
         }
 #pragma unroll
         for (int j = 0; j < kSegsPerStatsWarp; ++j) {
-            const int k = warp + j * kStatsWarps;
+            const int k = warp + j * NSW;
             if (k < ns) {
                 sh.fsum[k][lane] = ps[j];
                 sh.fmin[k][lane] = pn[j];
                 sh.fmax[k][lane] = px[j];
             }
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kStatsWarps * 32));
+        asm volatile("bar.sync 1, %0;" ::"n"(NSW * 32));
         if (warp == 0) {
             for (int k = 0; k < ns; ++k) {
                 S = __fadd_rn(S, sh.fsum[k][lane]);
@@ -430,7 +433,7 @@ __device__ float finalize_block(const QuantArgs& a, QuantShared& sh, int b) {
                 mx = fmaxf(mx, __uint_as_float((uint32_t)sh.fmax[k][lane] << 16));
             }
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kStatsWarps * 32));
+        asm volatile("bar.sync 1, %0;" ::"n"(NSW * 32));
     }
     float kp = 0.0f;
     if (warp == 0) {
@@ -549,7 +552,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
     volatile int* abort = &sh.abort;
     uint8_t* sbst = sh.sb[warp];
 
-    if (warp < kStatsWarps) {
+    constexpr int NSW = ROPE ? kStatsWarpsRope : kStatsWarps;
+    if (warp < NSW) {
         // 2a. K statistics from HBM
         int done = 0;
         for (int i; (i = take(&sh.q_stats, s1 - s0, abort)) >= 0; ++done)
@@ -563,9 +567,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
             // warp must not split them across the named barriers below)
             if (threadIdx.x == 0)
                 sh.fin_go = wait_counter(&a.ctl->q_sdone, (unsigned)n_stats, a.ctl, abort, 106u);
-            asm volatile("bar.sync 1, %0;" ::"n"(kStatsWarps * 32));
+            asm volatile("bar.sync 1, %0;" ::"n"(NSW * 32));
             if (!sh.fin_go) break;
-            const float kp = finalize_block(a, sh, fb);
+            const float kp = finalize_block<NSW>(a, sh, fb);
             if (warp == 0 && lane == 0) {
                 atomicMax(&a.ctl->q_kmax, __float_as_uint(kp));
                 __threadfence();
@@ -576,7 +580,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quantize_kernel(QuantArgs a)
     }
     // 2c. V from L2
     if (ensure_table(a, sh, 0)) {
-        if (warp == kStatsWarps && lane == 0) stamp(a, 3);
+        if (warp == NSW && lane == 0) stamp(a, 3);
         const EncodeConsts c = encode_consts(sh.s[0]);
         for (int i; (i = take(&sh.q_v, u1 - u0, abort)) >= 0;) {
             const int u = u0 + i;

@@ -21,9 +21,9 @@
 // Two kernels: the table of a chunk (one thread per entry), and the rotation
 // of a bf16 [T][H][128] tensor (the queries; the chunk quantizer rotates K
 // itself inside its statistics and encoding passes, quant.cu).  The rotation
-// moves 2 bytes in and 2 bytes out per element and is bound by HBM: two CTAs
-// per SM stage the table in shared memory (rope.cuh's padded rows), and each
-// thread keeps four 16-byte loads in flight.
+// moves 2 bytes in and 2 bytes out per element and is bound by HBM: a thread
+// takes 8 channels of one token in every head, reads their four table entries
+// once, and keeps 12 heads' 16-byte loads in flight.
 #include "common.cuh"
 #include "kernels.h"
 #include "rope.cuh"
@@ -55,41 +55,60 @@ __global__ void rope_table_kernel(long long frame_pos0, int frames, int rows, in
     }
 }
 
-constexpr int kRopeThreads = 512;
-constexpr int kRopeUnroll = 4;            // 16-byte loads in flight per thread
+constexpr int kRopeThreads = 256;
+constexpr int kRopeBatch = 12;            // heads whose 16-byte loads are in flight together
 
-// Units of 16 bytes: unit u of X is token (u / 16) / H, channels 8 q .. 8 q + 7
-// with q = u % 16 (head pairs 4 q .. 4 q + 3).  The grid stride is a multiple
-// of 16, so a thread keeps one q and one pair group.
+// Table entry of head pair P for a token at frame f, row r, column c.
+__device__ __forceinline__ int rope_entry(const RopeDev& g, int f, int r, int c, int P) {
+    if (P < kRopeRowPair0) return f * kRopeFramePairs + P;
+    if (P < kRopeColPair0) return g.frames * kRopeFramePairs + r * kRopeAxisPairs + P - kRopeRowPair0;
+    return g.frames * kRopeFramePairs + g.rows * kRopeAxisPairs + c * kRopeAxisPairs + P -
+           kRopeColPair0;
+}
+
+// Thread = (token t, channel group q): the 8 channels 8 q .. 8 q + 7 (head
+// pairs 4 q .. 4 q + 3) of every head of token t.  Their four table entries
+// depend on the token and the pairs only, so they are read once (through L1)
+// and kept in registers for all H heads; a warp covers two tokens, each head's
+// 256 bytes of a token contiguous.
 __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const uint4* X, uint4* Y, int T,
-                                                            int H, uint64_t m_h, RopeDev g) {
-    extern __shared__ float2 rope_sm[];
-    rope_stage(g, rope_sm);
-    __syncthreads();
-    const uint32_t n16 = (uint32_t)T * (uint32_t)H * 16u;
-    const uint32_t stride = gridDim.x * blockDim.x;
-    const uint32_t first = blockIdx.x * blockDim.x + threadIdx.x;
-    const RopeGroup grp = rope_group(4 * (int)(first & 15u));
-    for (uint32_t u0 = first; u0 < n16; u0 += kRopeUnroll * stride) {
-        uint4 w[kRopeUnroll];
+                                                            int H, RopeDev g) {
+    const int q = threadIdx.x & 15;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 4; t < T;
+         t += (gridDim.x * blockDim.x) >> 4) {
+        const uint4* src = X + (size_t)t * H * 16 + q;
+        uint4* dst = Y + (size_t)t * H * 16 + q;
+        uint4 w[kRopeBatch];
+        // the first heads' loads go out before the table reads they do not need
 #pragma unroll
-        for (int k = 0; k < kRopeUnroll; ++k) {
-            const uint32_t u = u0 + k * stride;
-            w[k] = u < n16 ? __ldcs(X + u) : make_uint4(0u, 0u, 0u, 0u);
-        }
+        for (int k = 0; k < kRopeBatch; ++k)
+            w[k] = k < H ? __ldcs(src + k * 16) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t f = rope_div((uint32_t)t, g.m_rc);
+        const uint32_t rem = (uint32_t)t - f * (uint32_t)g.rc;
+        const uint32_t r = rope_div(rem, g.m_c);
+        const uint32_t c = rem - r * (uint32_t)g.cols;
+        float2 cs[4];
 #pragma unroll
-        for (int k = 0; k < kRopeUnroll; ++k) {
-            const uint32_t u = u0 + k * stride;
-            if (u < n16) {
-                uint32_t v[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
-                rope_group4(grp, rope_rows(g, rope_div(u >> 4, m_h)), rope_sm, g.one, v);
-                __stcs(Y + u, make_uint4(v[0], v[1], v[2], v[3]));
+        for (int j = 0; j < 4; ++j) cs[j] = __ldg(g.tab + rope_entry(g, f, r, c, 4 * q + j));
+        for (int h0 = 0; h0 < H; h0 += kRopeBatch) {
+            if (h0 > 0) {
+#pragma unroll
+                for (int k = 0; k < kRopeBatch; ++k)
+                    w[k] = h0 + k < H ? __ldcs(src + (h0 + k) * 16) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < kRopeBatch; ++k) {
+                if (h0 + k < H) {
+                    const uint4 v = make_uint4(rope_pair(w[k].x, cs[0], g.one),
+                                               rope_pair(w[k].y, cs[1], g.one),
+                                               rope_pair(w[k].z, cs[2], g.one),
+                                               rope_pair(w[k].w, cs[3], g.one));
+                    __stcs(dst + (h0 + k) * 16, v);
+                }
             }
         }
     }
 }
-
-bool g_rope_smem_set[64];   // the dynamic shared memory limit raised, per device
 
 }  // namespace
 
@@ -128,23 +147,13 @@ nvfp4kv_status launch_rope_table(long long frame_pos0, int frames, int rows, int
 
 nvfp4kv_status launch_rope(const void* X, void* Y, int T, int H, const RopeGeom& r,
                            cudaStream_t stream) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4KV_ERR_CUDA;
-    if (!g_rope_smem_set[dev]) {
-        if (cudaFuncSetAttribute(rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kRopeMaxStagedBytes) != cudaSuccess)
-            return NVFP4KV_ERR_CUDA;
-        g_rope_smem_set[dev] = true;
-    }
     const int sms = sm_count_cached();
     if (sms <= 0) return NVFP4KV_ERR_CUDA;
-    const long long n16 = (long long)T * H * 16;
-    const long long per_pass = (long long)kRopeThreads * kRopeUnroll;
-    const long long want = (n16 + per_pass - 1) / per_pass;
-    const int blocks = (int)(want < 2LL * sms ? want : 2LL * sms);
-    rope_kernel<<<blocks, kRopeThreads, rope_staged_bytes(r.frames, r.rows, r.cols), stream>>>(
-        static_cast<const uint4*>(X), static_cast<uint4*>(Y), T, H,
-        rope_reciprocal((uint32_t)H), rope_dev(r));
+    const long long threads = 16LL * T;
+    const long long want = (threads + kRopeThreads - 1) / kRopeThreads;
+    const int blocks = (int)(want < 4LL * sms ? want : 4LL * sms);
+    rope_kernel<<<blocks, kRopeThreads, 0, stream>>>(static_cast<const uint4*>(X),
+                                                     static_cast<uint4*>(Y), T, H, rope_dev(r));
     return cudaGetLastError() == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 

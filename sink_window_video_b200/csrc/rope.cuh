@@ -37,27 +37,28 @@ __host__ __device__ inline int rope_staged_slots(int frames, int rows, int cols)
 }
 
 // Token geometry of a rotation: the table and the frame grid, with the
-// reciprocals m = floor(2^32 / D) + 1 of rows*cols and cols (33 bits for
-// D = 1), so that t / D = (t * m) >> 32 exactly whenever t * D < 2^32:
-// m D - 2^32 = e lies in (0, D], and t e < 2^32 keeps the fraction below 1.
+// reciprocals m = floor(2^32 / D) + 1 of rows*cols and cols, so that
+// t / D = umulhi(t, m) exactly whenever t * D < 2^32: m D - 2^32 = e lies in
+// (0, D], and t e < 2^32 keeps the fraction below 1.  D = 1 (m = 2^32 does
+// not fit) is marked by m = 0 and divides as t itself.
 struct RopeDev {
     const float2* tab;             // device table (entries above)
     int frames, rows, cols, rc;
     int entries;                   // frames*22 + (rows + cols)*21
     int rowslot, colslot;          // first staged slot of the row and column parts
-    uint64_t m_rc, m_c;
+    uint32_t m_rc, m_c;
     float one;                     // 1 as a run-time value (see rope_pair)
 };
 
 // The device view of a rotation's geometry (rope.cu).
 RopeDev rope_dev(const RopeGeom& r);
 
-__host__ __device__ inline uint64_t rope_reciprocal(uint32_t D) {
-    return (1ull << 32) / D + 1ull;
+__host__ __device__ inline uint32_t rope_reciprocal(uint32_t D) {
+    return D > 1 ? (uint32_t)((1ull << 32) / D + 1ull) : 0u;
 }
 
-__device__ __forceinline__ uint32_t rope_div(uint32_t t, uint64_t m) {
-    return (uint32_t)(((uint64_t)t * m) >> 32);
+__device__ __forceinline__ uint32_t rope_div(uint32_t t, uint32_t m) {
+    return m ? __umulhi(t, m) : t;
 }
 
 // Copy the table into shared memory sm (rope_staged_slots float2), every
@@ -129,16 +130,17 @@ __device__ __forceinline__ int rope_row_of(const RopeRows& b, int part) {
 // One bf16 channel pair u = (x0 low half, x1 high half) turned by the entry
 // {cos, sin}: (x0 cos - x1 sin, x1 cos + x0 sin), one fp32 rounding per
 // product and per sum, each result rounded to bf16 (RN-even).  The sums are
-// fma(b, (-one, one), a) with `one` a run-time 1 (b * -1 and b * 1 are exact):
-// a separate paired multiply and add may be fused by the compiler into one
+// fma(product, -+one, product) with `one` a run-time 1 (p * -1 and p * 1 are
+// exact): a separate multiply and add may be fused by the compiler into one
 // fma, which skips the rounding of a product (and moves results that sit on a
 // bf16 tie); a multiply cannot be merged into the multiplicand of an fma.
 __device__ __forceinline__ uint32_t rope_pair(uint32_t u, float2 cs, float one) {
     const float2 x = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-    const float2 a = __fmul2_rn(x, make_float2(cs.x, cs.x));
-    const float2 b = __fmul2_rn(make_float2(x.y, x.x), make_float2(cs.y, cs.y));
-    const float2 y = __ffma2_rn(b, make_float2(-one, one), a);
-    const __nv_bfloat162 r = __floats2bfloat162_rn(y.x, y.y);
+    const float2 a = __fmul2_rn(x, make_float2(cs.x, cs.x));      // x0 cos, x1 cos
+    const float2 b = __fmul2_rn(x, make_float2(cs.y, cs.y));      // x0 sin, x1 sin
+    const float y0 = __fmaf_rn(b.y, -one, a.x);
+    const float y1 = __fmaf_rn(b.x, one, a.y);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(y0, y1);
     return *reinterpret_cast<const uint32_t*>(&r);
 }
 
