@@ -56,7 +56,7 @@ NCU_TRAFFIC = {
     "matrix_1d": ("sink_window_video_b200/csrc/matrix_quant.cu",
                   "3286f4378a02393756ca9d2ec0164e9ec70777adf69cdacefd0d340704548b10", 43654912),
     "quantize": ("sink_window_video_b200/csrc/quant.cu",
-                 "ffba28cf4e3a2bc13d72d317f9f51162afdaa58cb295fff9792e1e3d0661758e", 98012416),
+                 "6a3a95c215cb0d9dd447332b23b0bcaf29d066650881108d9bb1c8938d060cfa", 97882112),
     "attention_fp4": ("sink_window_video_b200/csrc/attention_fp4.cu",
                       "385b563baf2156d9f340a5b351f880de978d2ecddd7e92a3ddefc57bd36f4a2b", 194231296),
     "rope": ("sink_window_video_b200/csrc/rope.cu",
