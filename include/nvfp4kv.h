@@ -14,6 +14,10 @@
  *     A_s over K_eff(t) = A_g u A_s u KV[t-W, t), overlapping tokens counted
  *     once, A_s tracked by two pointers and re-bound on a prompt switch
  *     (DeepRead page, Method > 算法层设计, Multi-Shot Attention Sink).
+ *   - a 3D rotary position embedding of queries and keys with the multi-shot
+ *     frame offset, fused into the quantizer for K (txtmix page "LongLive 2.0：
+ *     给长视频生成补上 NVFP4 并行基础设施", sections NVFP4 and 多 shot 一致性;
+ *     the rotary form is a stated reading, see the rotary section below).
  *
  * Conventions for every entry point:
  *   - "device" pointers are CUDA device memory owned by the CALLER (for
