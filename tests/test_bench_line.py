@@ -17,6 +17,9 @@ def _measurements(e2e=True, extras=True):
         r["rollouts"] = [{"workload": "w", "chunks_per_s": 11.0, "frac": 0.66}]
         r["matrix"] = [{"workload": "m", "us_per_launch": 42.0}]
         r["dequant"] = {"kernel": "d", "us_per_launch": 27.0}
+        r["rope"] = {"workload": "r", "table_us": 8.0,
+                     "rope": {"us_per_launch": 17.0, "frac": 0.77},
+                     "quantize_rope": {"us_per_launch": 80.0, "unfused_us": 75.0}}
     return r
 
 
@@ -45,7 +48,7 @@ def test_line_has_the_contract_keys(world):
     e = line["e2e"]
     assert e["unit"] == line["unit"] and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert line["gpu_launches"] == 300 * 3
-    for k in ("rollouts", "matrix_quantize", "dequantize", "quantize", "attention"):
+    for k in ("rollouts", "matrix_quantize", "dequantize", "quantize", "attention", "rope"):
         assert k in line
     json.dumps(line)
 
@@ -54,7 +57,7 @@ def test_line_without_optional_parts():
     import bench
     args = types.SimpleNamespace(steps=20, warmup=3)
     line = bench.build_line(args, _measurements(e2e=False, extras=False), 1, {}, "fallback")
-    for k in ("e2e", "rollouts", "matrix_quantize", "dequantize"):
+    for k in ("e2e", "rollouts", "matrix_quantize", "dequantize", "rope"):
         assert k not in line
     json.dumps(line)
 
