@@ -126,8 +126,8 @@ struct RopeGeom {
     int frames, rows, cols;
 };
 size_t rope_table_entries(int frames, int rows, int cols);
-// Shared memory of a staged table (rope.cuh's padded rows); kernels that stage
-// it take grids up to kRopeMaxStagedBytes.
+// Shared memory of a staged table (rope.cuh's padded rows, the chunk
+// quantizer's copy); the entry points accept grids up to kRopeMaxStagedBytes.
 constexpr size_t kRopeMaxStagedBytes = 61440;
 size_t rope_staged_bytes(int frames, int rows, int cols);
 nvfp4kv_status launch_rope_table(long long frame_pos0, int frames, int rows, int cols,

@@ -9,10 +9,11 @@
 // Head channels (d = 128): frame pairs 0..21 (channels 0..43), row pairs
 // 22..42 (44..85), column pairs 43..63 (86..127).
 //
-// The consuming kernels stage the table in shared memory, one row per
+// The chunk quantizer stages the table in shared memory, one row per
 // coordinate with head pair P at slot P + P/4 (less the part's first slot):
 // lanes that take head pairs 4 apart then read different banks, and the four
-// pairs of an aligned group P0..P0+3 sit in consecutive slots.
+// pairs of an aligned group P0..P0+3 sit in consecutive slots.  rope_kernel
+// reads its few entries per token straight from the device table.
 #pragma once
 
 #include <cuda_bf16.h>
