@@ -231,7 +231,8 @@ nvfp4kv_status nvfp4kv_rope_table(long long frame_pos0, int frames, int rows, in
 
 /* Rotate X ([T][H][d] bf16, device) into Y (same layout; Y == X rotates in
  * place, other overlaps are not allowed): the queries of a chunk whose keys go
- * through nvfp4kv_quantize_chunk_rope with the same table.  T <= 65535,
+ * through nvfp4kv_quantize_chunk_rope with the same table; a partial overlap
+ * is refused with NVFP4KV_ERR_INVALID_ARG.  T <= 65535,
  * T*H*H < 2^32, frames*rows*cols >= T, and the table small enough to stage in
  * shared memory: 8 * (27*frames + 26*(rows + cols)) <= 61440 bytes
  * (NVFP4KV_ERR_INVALID_ARG otherwise).  One launch; bound by HBM (2 bytes

@@ -256,6 +256,13 @@ nvfp4kv_status nvfp4kv_rope(const void* X, void* Y, int T, int H, int d,
                             const nvfp4kv_rope_view* rope, nvfp4kv_stream_t stream) {
     if (!X || !Y || !valid_shape(T, H, d) || (long long)T * H * H >= (1LL << 32))
         return NVFP4KV_ERR_INVALID_ARG;
+    {
+        // Y == X rotates in place (each 16 bytes read and written by one
+        // thread); any other overlap would let a write land before a read
+        const uintptr_t x0 = reinterpret_cast<uintptr_t>(X), y0 = reinterpret_cast<uintptr_t>(Y);
+        const uintptr_t n = (uintptr_t)T * H * d * 2;
+        if (x0 != y0 && x0 < y0 + n && y0 < x0 + n) return NVFP4KV_ERR_INVALID_ARG;
+    }
     const nvfp4kv_status st = check_rope_view(rope, T);
     if (st != NVFP4KV_OK) return st;
     if (d != kHeadDimSupported) return NVFP4KV_ERR_UNSUPPORTED;

@@ -377,7 +377,13 @@ def test_rope_entry_points_refuse_bad_arguments(L):
     assert L.nvfp4kv_rope(FAKE, FAKE, 7041, 24, 128, r, None) == swv.ERR_INVALID_ARG  # > 8 frames
     assert L.nvfp4kv_rope(FAKE, FAKE, 0, 24, 128, r, None) == swv.ERR_INVALID_ARG
     assert L.nvfp4kv_rope(FAKE, FAKE, 7040, 24, 96, r, None) == swv.ERR_UNSUPPORTED
-    assert L.nvfp4kv_rope(FAKE + 8, FAKE, 7040, 24, 128, r, None) == swv.ERR_ALIGNMENT
+    n = 7040 * 24 * 128 * 2
+    for y in (FAKE + 16, FAKE + n - 16, FAKE - n + 16):                 # partial overlaps
+        assert L.nvfp4kv_rope(FAKE, y, 7040, 24, 128, r, None) == swv.ERR_INVALID_ARG
+    for y in (FAKE, FAKE + n, FAKE - n):                                 # in place, disjoint
+        assert L.nvfp4kv_rope(FAKE, y, 7040, 24, 128, r, None) == swv.ERR_UNSUPPORTED
+    far = FAKE + (1 << 32)                                      # disjoint from X
+    assert L.nvfp4kv_rope(FAKE + 8, far, 7040, 24, 128, r, None) == swv.ERR_ALIGNMENT
     assert L.nvfp4kv_rope(FAKE, FAKE, 100, 1 << 13, 128, r, None) == swv.ERR_INVALID_ARG
     big = swv.RopeView(FAKE, 2, 300, 300)                       # rows * cols > 65535
     assert L.nvfp4kv_rope(FAKE, FAKE, 100, 2, 128, ctypes.byref(big), None) == \
